@@ -1,0 +1,242 @@
+/*
+ * sfc.h -- C ABI of libsfc: self-synchronizing small-message all-reduce and
+ * all-gather with N ranks emulated inside one B200.
+ *
+ * What is computed ("flash-comm: Self-Synchronizing Collective Communication
+ * for LLM Decoding", abstract): an all-reduce in which every data block
+ * carries its own readiness evidence, so a receiver validates exactly the
+ * blocks it needs and no separate barrier is run; the reduction order is
+ * fixed (rank 0, 1, ..., N-1, fp32 accumulation, one rounding to bf16) and
+ * independent of the order in which blocks arrive, so every rank gets the
+ * same bits; the same mechanism gives a standalone all-gather.
+ *
+ * Readiness encodings ("Why Microseconds Matter in AI Infrastructure",
+ * section "Latency can matter more than bandwidth"):
+ *   LL       -- data and flag in one atomic store: each 8-byte unit holds two
+ *               bf16 elements and the 32-bit epoch.
+ *   LL128    -- a 128-byte line of 120 data bytes and an 8-byte epoch flag.
+ *   SENTINEL -- raw data into a receive buffer pre-filled with the negative
+ *               NaN 0xFFFF, polled until it changes, then reset.
+ * Double buffering by epoch parity (same section) replaces the bottom barrier.
+ * The explicit-barrier oneshot / twoshot algorithms ("SiFAR:
+ * Synchronization-Free All-Reduce for Low-Latency LLM Inference", abstract)
+ * are provided in the same kernel framework as the comparison baseline.
+ *
+ * Emulation: rank r is a group of co-resident CTAs of one persistent
+ * cooperative kernel; "sending to rank p" is a store into rank p's scratch in
+ * this GPU's HBM. No data crosses a GPU boundary.
+ *
+ * Conventions shared by every call:
+ *   - Pointers named "device" are CUDA device pointers on the context's
+ *     device; pointers named "host" are host pointers. Tensor data is bf16
+ *     (raw 16-bit patterns), element counts are per rank.
+ *   - in[r] / out[r] are owned by the caller, 16-byte aligned, and must not
+ *     overlap each other (no in-place). The library never reads an input
+ *     after the call's kernel has finished and never writes an input.
+ *   - Epochs: 32-bit, start at 1 after sfc_init / sfc_reset; every
+ *     operation consumes one, and a call must pass exactly the next one
+ *     (sfc_next_epoch), else SFC_ERR_EPOCH. All-reduce and all-gather share
+ *     the sequence. Parity = epoch & 1 selects the scratch buffer.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*,
+ *     NULL = the legacy default stream). Calls on one context must be
+ *     ordered on the GPU (one stream, or streams joined by events).
+ *   - Device-side errors (a wait that ran out, a sentinel in an input under
+ *     debug checks) are sticky: the kernel records them and every later
+ *     kernel of the context exits at once, until sfc_reset. They are read
+ *     with sfc_get_status.
+ */
+#ifndef SFC_H
+#define SFC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct sfc_ctx sfc_ctx;
+
+typedef enum {
+  SFC_OK = 0,
+  SFC_ERR_INVALID = 1,            /* bad argument; nothing was launched */
+  SFC_ERR_CUDA = 2,               /* a CUDA runtime call failed */
+  SFC_ERR_TIMEOUT = 3,            /* a device wait exceeded timeout_us */
+  SFC_ERR_EPOCH = 4,              /* epoch is not the next one */
+  SFC_ERR_RESOURCES = 5,          /* the ranks' CTAs cannot all be co-resident */
+  SFC_ERR_SENTINEL_IN_INPUT = 6,  /* input holds 0xFFFF (debug checks only) */
+  SFC_ERR_UNSUPPORTED = 7,        /* protocol / op / dtype combination not provided */
+  SFC_ERR_ABORTED = 8             /* context poisoned by an earlier device error */
+} sfc_status;
+
+typedef enum {
+  SFC_PROTO_AUTO = 0,             /* ask the selector */
+  SFC_PROTO_LL = 1,
+  SFC_PROTO_LL128 = 2,
+  SFC_PROTO_SENTINEL = 3,
+  SFC_PROTO_BARRIER_ONESHOT = 4,  /* pull, top + bottom barrier */
+  SFC_PROTO_BARRIER_TWOSHOT = 5   /* all-reduce only: reduce-scatter + all-gather */
+} sfc_protocol;
+
+#define SFC_NUM_PROTOCOLS 6
+#define SFC_MAX_RANKS 8
+
+typedef enum { SFC_BF16 = 0 } sfc_dtype;
+
+typedef enum { SFC_OP_ALLREDUCE = 0, SFC_OP_ALLGATHER = 1 } sfc_op;
+
+typedef struct {
+  int ctas_per_rank;        /* CTAs per emulated rank; 0 = chosen per call */
+  uint32_t timeout_us;      /* bound on each device-side wait; 0 = 50000 */
+  int debug_checks;         /* nonzero: the kernel rejects sentinel inputs */
+  uint32_t protocol_mask;   /* bit p provisions scratch for protocol p; 0 = all */
+} sfc_config;
+
+/* Latency model of the selector: T = alpha_us + beta_us_per_byte * bytes,
+ * bytes = sfc_algorithmic_bytes(op, protocol, count, nranks). An entry with
+ * alpha_us < 0 marks the protocol unavailable for that rank count. */
+typedef struct {
+  double alpha_us;
+  double beta_us_per_byte;
+} sfc_cost_coeff;
+
+typedef struct {
+  sfc_cost_coeff c[2][SFC_NUM_PROTOCOLS][SFC_MAX_RANKS + 1]; /* [op][protocol][nranks] */
+} sfc_cost_model;
+
+typedef struct {
+  double flag_rtt_ns_p50;   /* two CTAs on different SMs ping-pong a flag */
+  double flag_rtt_ns_p99;
+  double l2_rtt_ns_p50;     /* dependent L2-hit loads, one thread */
+  double sm_clock_ghz;      /* clock64 ticks per globaltimer ns during the run */
+  double globaltimer_step_ns; /* smallest nonzero globaltimer increment seen */
+  int sm_a, sm_b;           /* SMs the two ping-pong CTAs ran on (last trial) */
+} sfc_floor_result;
+
+/* Create a context for `nranks` (2..8) emulated ranks on the current CUDA
+ * device, with scratch for messages up to `max_bytes_per_rank` bytes per rank
+ * (all-gather: per shard). Allocates the scratch (per provisioned protocol:
+ * 2 parities x N x (N-1) encoded slots), barrier flags and status words;
+ * sentinel slots are filled with 0xFFFF, flags zeroed, next epoch = 1.
+ * cfg may be NULL (defaults). Synchronous. */
+sfc_status sfc_init(sfc_ctx** ctx, int nranks, size_t max_bytes_per_rank, const sfc_config* cfg);
+
+/* Free everything the context owns (synchronizes the device first). */
+sfc_status sfc_destroy(sfc_ctx* ctx);
+
+/* Return the context to its initial state on `stream`: refill sentinel
+ * slots, zero flags and barrier counters, clear the sticky error; the next
+ * epoch becomes 1. The only way out of a device error. */
+sfc_status sfc_reset(sfc_ctx* ctx, void* stream);
+
+/* One all-reduce. in/out: HOST arrays of N DEVICE pointers, each to `count`
+ * bf16 elements. After the kernel, out[r][i] = bf16_RNE(sum over q = 0..N-1,
+ * in rank order, of fp32(in[q][i])) for every rank r. count == 0 is a no-op
+ * that consumes no epoch. protocol AUTO asks the selector. */
+sfc_status sfc_allreduce(sfc_ctx* ctx, const void* const* in, void* const* out, size_t count,
+                         sfc_dtype dtype, sfc_protocol protocol, uint32_t epoch, void* stream);
+
+/* One all-gather. in: N device pointers to `count` elements; out: N device
+ * pointers to N*count elements; out[r] = in[0] || in[1] || ... || in[N-1].
+ * BARRIER_TWOSHOT is not an all-gather algorithm (SFC_ERR_UNSUPPORTED). */
+sfc_status sfc_allgather(sfc_ctx* ctx, const void* const* in, void* const* out, size_t count,
+                         sfc_dtype dtype, sfc_protocol protocol, uint32_t epoch, void* stream);
+
+/* k_ops operations issued back to back inside ONE persistent launch,
+ * epochs first_epoch .. first_epoch + k_ops - 1 (the decode step's chain of
+ * per-layer all-reduces). in_table / out_table: DEVICE arrays of k_ops*N
+ * device pointers, entry [k*N + r] for operation k, rank r. No input may be
+ * an output of the same chain. skew_ns: DEVICE array [k_ops*N] or NULL;
+ * before pushing operation k, rank r spins skew_ns[k*N + r] ns (capped at
+ * the timeout). timings: DEVICE array [k_ops + 1] or NULL; the library
+ * clears it on `stream`, then timings[0] = earliest kernel start and
+ * timings[1 + k] = latest completion of operation k over all warps, in
+ * %globaltimer nanoseconds. */
+sfc_status sfc_allreduce_chain(sfc_ctx* ctx, int k_ops, const void* const* in_table,
+                               void* const* out_table, size_t count, sfc_dtype dtype,
+                               sfc_protocol protocol, uint32_t first_epoch,
+                               const uint32_t* skew_ns, uint64_t* timings, void* stream);
+
+/* The all-gather counterpart of sfc_allreduce_chain (out entries hold
+ * N*count elements). */
+sfc_status sfc_allgather_chain(sfc_ctx* ctx, int k_ops, const void* const* in_table,
+                               void* const* out_table, size_t count, sfc_dtype dtype,
+                               sfc_protocol protocol, uint32_t first_epoch,
+                               const uint32_t* skew_ns, uint64_t* timings, void* stream);
+
+/* End-to-end all-reduce chain from HOST memory: in_host holds
+ * [k_ops][N][count] bf16 contiguous, out_host receives [k_ops][N][count].
+ * Copies the inputs to context-owned device staging (allocated on first use,
+ * grown as needed), runs the chain, copies the outputs back, all on
+ * `stream`; the call returns once the copies are queued. Page-locked host
+ * memory makes the copies asynchronous. timings as in sfc_allreduce_chain. */
+sfc_status sfc_allreduce_chain_host(sfc_ctx* ctx, int k_ops, const void* in_host, void* out_host,
+                                    size_t count, sfc_dtype dtype, sfc_protocol protocol,
+                                    uint32_t first_epoch, uint64_t* timings, void* stream);
+
+/* The selector (cost-guided choice of the encoding by message size and rank
+ * count: "flash-comm: Self-Synchronizing Collective Communication for LLM
+ * Decoding", abstract; the empirical choice in "Why Microseconds Matter in AI
+ * Infrastructure", section "What I learned from it"). argmin over protocols
+ * of alpha + beta * bytes; ties go to fewer bytes, then to the order
+ * SENTINEL, LL128, LL, BARRIER_ONESHOT, BARRIER_TWOSHOT. Host only. */
+sfc_protocol sfc_select_protocol(const sfc_ctx* ctx, sfc_op op, size_t bytes_per_rank, int nranks);
+
+/* The same choice from an explicit model; needs no context and no GPU. */
+sfc_protocol sfc_select_protocol_model(const sfc_cost_model* model, sfc_op op,
+                                       size_t bytes_per_rank, int nranks);
+
+/* Replace the context's model (copied). The built-in default comes from a
+ * fit on B200 measurements. */
+sfc_status sfc_set_cost_model(sfc_ctx* ctx, const sfc_cost_model* model);
+
+/* Write the built-in default model into *model. */
+void sfc_default_cost_model(sfc_cost_model* model);
+
+/* Algorithmic bytes of one operation summed over all ranks (encoded bytes
+ * written plus bytes read; the sentinel's reset writes included); the
+ * roofline numerator. Returns -1 for an unsupported combination. */
+double sfc_algorithmic_bytes(sfc_op op, sfc_protocol protocol, size_t count, int nranks);
+
+/* Synchronize the context's last stream and return its sticky device status
+ * (SFC_OK if none). *info (may be NULL) receives detail: for a timeout,
+ * (operation index << 16) | (rank << 8) | source. The error stays set until
+ * sfc_reset. */
+sfc_status sfc_get_status(sfc_ctx* ctx, uint32_t* info);
+
+/* Static English name of a status. */
+const char* sfc_status_string(sfc_status s);
+
+/* The epoch the next operation must use. */
+uint32_t sfc_next_epoch(const sfc_ctx* ctx);
+
+/* The launch shape a call would use: CTAs per rank and threads per CTA. */
+sfc_status sfc_launch_shape(sfc_ctx* ctx, sfc_op op, sfc_protocol protocol, size_t count,
+                            int* ctas_per_rank, int* threads_per_cta);
+
+/* Device address and byte size of one receive slot of the scratch, for
+ * inspection by tests: rank `rank`'s slot for source `src` (!= rank) at
+ * `parity`, under `protocol` (LL, LL128 or SENTINEL). */
+sfc_status sfc_scratch_slot(sfc_ctx* ctx, sfc_protocol protocol, int rank, int parity, int src,
+                            void** device_ptr, size_t* bytes);
+
+/* Fault injection on the host side: from the next launch on, rank
+ * `silent_rank` pushes nothing and arrives at no barrier (-1 = off). Its
+ * peers' waits then run out after timeout_us and report SFC_ERR_TIMEOUT. */
+sfc_status sfc_set_silent_rank(sfc_ctx* ctx, int silent_rank);
+
+/* Latency floor microbenchmarks on the current device (synchronous, owns
+ * its buffers): a flag round trip between two CTAs on different SMs and the
+ * L2 hit latency. The speed-of-light bound of "Why Microseconds Matter in AI
+ * Infrastructure", section "Defining the physical lower bound", is built
+ * from such round trips. iters >= 16. */
+sfc_status sfc_measure_floor(int iters, sfc_floor_result* out);
+
+/* Number of kernel launches this context has issued (all entry points). */
+uint64_t sfc_launch_count(const sfc_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SFC_H */

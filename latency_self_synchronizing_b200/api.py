@@ -1,0 +1,273 @@
+"""Python binding over libsfc: torch tensors and streams in, C ABI calls out.
+
+Every step of the collective runs in the CUDA library; this module only
+checks tensor metadata, collects device pointers and the current stream, and
+turns status codes into exceptions.
+"""
+
+import ctypes as C
+import enum
+
+import torch
+
+from . import _lib
+
+__all__ = [
+    "Status", "Protocol", "Op", "SfcError", "Communicator", "pointer_table", "measure_floor",
+    "algorithmic_bytes", "select_protocol_model", "default_cost_model", "status_string",
+]
+
+
+class Status(enum.IntEnum):
+    OK = 0
+    INVALID = 1
+    CUDA = 2
+    TIMEOUT = 3
+    EPOCH = 4
+    RESOURCES = 5
+    SENTINEL_IN_INPUT = 6
+    UNSUPPORTED = 7
+    ABORTED = 8
+
+
+class Protocol(enum.IntEnum):
+    AUTO = 0
+    LL = 1
+    LL128 = 2
+    SENTINEL = 3
+    BARRIER_ONESHOT = 4
+    BARRIER_TWOSHOT = 5
+
+
+class Op(enum.IntEnum):
+    ALLREDUCE = 0
+    ALLGATHER = 1
+
+
+_NAMES = {"auto": Protocol.AUTO, "ll": Protocol.LL, "ll128": Protocol.LL128, "sentinel": Protocol.SENTINEL,
+          "barrier_oneshot": Protocol.BARRIER_ONESHOT, "oneshot": Protocol.BARRIER_ONESHOT,
+          "barrier_twoshot": Protocol.BARRIER_TWOSHOT, "twoshot": Protocol.BARRIER_TWOSHOT}
+
+
+def as_protocol(p):
+    if isinstance(p, str):
+        return _NAMES[p.lower()]
+    return Protocol(int(p))
+
+
+def as_op(o):
+    if isinstance(o, str):
+        return {"allreduce": Op.ALLREDUCE, "allgather": Op.ALLGATHER}[o.lower()]
+    return Op(int(o))
+
+
+class SfcError(RuntimeError):
+    def __init__(self, status, what=""):
+        self.status = Status(status)
+        super().__init__(f"{what}: {status_string(status)} ({self.status.name})")
+
+
+def status_string(s):
+    return _lib.load().sfc_status_string(int(s)).decode()
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise SfcError(rc, what)
+
+
+def _stream_handle(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+def _dev_ptr(t, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def pointer_table(rows):
+    """[[tensor per rank] per operation] -> int64 CUDA tensor of data pointers."""
+    ptrs = [_dev_ptr(t, "chain operand") for row in rows for t in row]
+    dev = rows[0][0].device
+    return torch.tensor(ptrs, dtype=torch.int64, device=dev)
+
+
+class Communicator:
+    """N emulated ranks on the current CUDA device (one libsfc context)."""
+
+    def __init__(self, nranks, max_bytes_per_rank, *, ctas_per_rank=0, timeout_us=0, debug_checks=False,
+                 protocols=None):
+        if not torch.cuda.is_available():
+            raise RuntimeError("a CUDA device is required")
+        self._lib = _lib.load()
+        mask = 0
+        if protocols is not None:
+            for p in protocols:
+                mask |= 1 << int(as_protocol(p))
+        cfg = _lib.Config(int(ctas_per_rank), int(timeout_us), int(bool(debug_checks)), mask)
+        handle = C.c_void_p()
+        torch.cuda.init()
+        _check(self._lib.sfc_init(C.byref(handle), int(nranks), int(max_bytes_per_rank), C.byref(cfg)), "sfc_init")
+        self._ctx = handle
+        self.nranks = int(nranks)
+        self.max_bytes_per_rank = int(max_bytes_per_rank)
+
+    # ----------------------------------------------------------- lifecycle
+    def close(self):
+        if getattr(self, "_ctx", None):
+            self._lib.sfc_destroy(self._ctx)
+            self._ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    @property
+    def next_epoch(self):
+        return int(self._lib.sfc_next_epoch(self._ctx))
+
+    def reset(self, stream=None):
+        _check(self._lib.sfc_reset(self._ctx, _stream_handle(stream)), "sfc_reset")
+
+    def status(self):
+        """(Status, info) after synchronizing the last stream used."""
+        info = C.c_uint32(0)
+        rc = self._lib.sfc_get_status(self._ctx, C.byref(info))
+        return Status(rc), int(info.value)
+
+    @property
+    def launch_count(self):
+        return int(self._lib.sfc_launch_count(self._ctx))
+
+    # --------------------------------------------------------- collectives
+    def _one(self, fn, op, inputs, outputs, protocol, epoch, stream):
+        n = self.nranks
+        if len(inputs) != n or len(outputs) != n:
+            raise ValueError(f"need {n} inputs and {n} outputs")
+        count = inputs[0].numel()
+        for t in inputs:
+            if t.numel() != count:
+                raise ValueError("all inputs must have the same number of elements")
+        want_out = count if op == Op.ALLREDUCE else n * count
+        for t in outputs:
+            if t.numel() != want_out:
+                raise ValueError(f"outputs must have {want_out} elements")
+        ins = (C.c_void_p * n)(*[_dev_ptr(t, "input") for t in inputs])
+        outs = (C.c_void_p * n)(*[_dev_ptr(t, "output") for t in outputs])
+        e = self.next_epoch if epoch is None else int(epoch)
+        _check(fn(self._ctx, ins, outs, count, 0, int(as_protocol(protocol)), e, _stream_handle(stream)),
+               fn.__name__)
+
+    def allreduce(self, inputs, outputs, protocol="auto", epoch=None, stream=None):
+        """outputs[r] = rank-order fp32 sum of inputs, rounded once to bf16."""
+        self._one(self._lib.sfc_allreduce, Op.ALLREDUCE, inputs, outputs, protocol, epoch, stream)
+
+    def allgather(self, inputs, outputs, protocol="auto", epoch=None, stream=None):
+        """outputs[r] = inputs[0] || ... || inputs[N-1]."""
+        self._one(self._lib.sfc_allgather, Op.ALLGATHER, inputs, outputs, protocol, epoch, stream)
+
+    def _chain(self, fn, in_table, out_table, count, k_ops, protocol, epoch, skew_ns, timings, stream):
+        n = self.nranks
+        for name, t in (("in_table", in_table), ("out_table", out_table)):
+            if t.dtype != torch.int64 or not t.is_cuda or t.numel() != k_ops * n:
+                raise ValueError(f"{name} must be an int64 CUDA tensor of {k_ops * n} pointers")
+        skew_p = None
+        if skew_ns is not None:
+            if skew_ns.dtype not in (torch.int32, torch.uint32) or skew_ns.numel() != k_ops * n:
+                raise ValueError("skew_ns must be an int32 CUDA tensor of k_ops * N entries")
+            skew_p = C.c_void_p(skew_ns.data_ptr())
+        tim_p = None
+        if timings is not None:
+            if timings.dtype != torch.int64 or timings.numel() < k_ops + 1:
+                raise ValueError("timings must be an int64 CUDA tensor of k_ops + 1 entries")
+            tim_p = C.c_void_p(timings.data_ptr())
+        e = self.next_epoch if epoch is None else int(epoch)
+        _check(fn(self._ctx, int(k_ops), C.c_void_p(in_table.data_ptr()), C.c_void_p(out_table.data_ptr()),
+                  int(count), 0, int(as_protocol(protocol)), e, skew_p, tim_p, _stream_handle(stream)),
+               fn.__name__)
+
+    def allreduce_chain(self, in_table, out_table, count, k_ops, protocol="auto", epoch=None, skew_ns=None,
+                        timings=None, stream=None):
+        """k_ops all-reduces in one persistent launch (pointer tables [k * N])."""
+        self._chain(self._lib.sfc_allreduce_chain, in_table, out_table, count, k_ops, protocol, epoch, skew_ns,
+                    timings, stream)
+
+    def allgather_chain(self, in_table, out_table, count, k_ops, protocol="auto", epoch=None, skew_ns=None,
+                        timings=None, stream=None):
+        self._chain(self._lib.sfc_allgather_chain, in_table, out_table, count, k_ops, protocol, epoch, skew_ns,
+                    timings, stream)
+
+    def allreduce_chain_host(self, in_host, out_host, protocol="auto", epoch=None, timings=None, stream=None):
+        """End to end from host memory: in_host / out_host are [k, N, count] bf16 CPU tensors."""
+        for name, t in (("in_host", in_host), ("out_host", out_host)):
+            if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 3:
+                raise ValueError(f"{name} must be a contiguous [k, N, count] bf16 CPU tensor")
+        k, n, count = in_host.shape
+        if n != self.nranks or tuple(out_host.shape) != (k, n, count):
+            raise ValueError("shape mismatch")
+        tim_p = None if timings is None else C.c_void_p(timings.data_ptr())
+        e = self.next_epoch if epoch is None else int(epoch)
+        _check(self._lib.sfc_allreduce_chain_host(self._ctx, int(k), C.c_void_p(in_host.data_ptr()),
+                                                  C.c_void_p(out_host.data_ptr()), int(count), 0,
+                                                  int(as_protocol(protocol)), e, tim_p, _stream_handle(stream)),
+               "sfc_allreduce_chain_host")
+
+    # ------------------------------------------------------------- helpers
+    def select_protocol(self, op, bytes_per_rank, nranks=None):
+        n = self.nranks if nranks is None else int(nranks)
+        return Protocol(self._lib.sfc_select_protocol(self._ctx, int(as_op(op)), int(bytes_per_rank), n))
+
+    def set_cost_model(self, model):
+        _check(self._lib.sfc_set_cost_model(self._ctx, C.byref(model)), "sfc_set_cost_model")
+
+    def launch_shape(self, op, protocol, count):
+        g, t = C.c_int(0), C.c_int(0)
+        _check(self._lib.sfc_launch_shape(self._ctx, int(as_op(op)), int(as_protocol(protocol)), int(count),
+                                          C.byref(g), C.byref(t)), "sfc_launch_shape")
+        return g.value, t.value
+
+    def scratch_slot(self, protocol, rank, parity, src):
+        """(device pointer, bytes) of one receive slot, for inspection."""
+        ptr, nb = C.c_void_p(), C.c_size_t()
+        _check(self._lib.sfc_scratch_slot(self._ctx, int(as_protocol(protocol)), int(rank), int(parity),
+                                          int(src), C.byref(ptr), C.byref(nb)), "sfc_scratch_slot")
+        return ptr.value, nb.value
+
+    def set_silent_rank(self, rank):
+        _check(self._lib.sfc_set_silent_rank(self._ctx, int(rank)), "sfc_set_silent_rank")
+
+
+def algorithmic_bytes(op, protocol, count, nranks):
+    return float(_lib.load().sfc_algorithmic_bytes(int(as_op(op)), int(as_protocol(protocol)), int(count),
+                                                   int(nranks)))
+
+
+def default_cost_model():
+    m = _lib.CostModel()
+    _lib.load().sfc_default_cost_model(C.byref(m))
+    return m
+
+
+def select_protocol_model(model, op, bytes_per_rank, nranks):
+    return Protocol(_lib.load().sfc_select_protocol_model(C.byref(model), int(as_op(op)), int(bytes_per_rank),
+                                                          int(nranks)))
+
+
+def measure_floor(iters=20000):
+    r = _lib.FloorResult()
+    _check(_lib.load().sfc_measure_floor(int(iters), C.byref(r)), "sfc_measure_floor")
+    return {f: getattr(r, f) for f, _ in _lib.FloorResult._fields_}

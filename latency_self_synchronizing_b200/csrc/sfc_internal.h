@@ -1,0 +1,84 @@
+// Internal definitions shared by the host runtime and the kernels of libsfc.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+namespace sfc {
+
+constexpr int kThreads = 256;  // threads per CTA of every collective kernel
+constexpr int kMaxRanks = 8;
+constexpr int kMinRanks = 2;
+
+// protocol ids (match sfc_protocol)
+enum : int { kLL = 1, kLL128 = 2, kSentinel = 3, kOneshot = 4, kTwoshot = 5 };
+// operations (match sfc_op)
+enum : int { kAllreduce = 0, kAllgather = 1 };
+
+// Barrier counter values are (epoch << 2) | phase, monotone over the whole
+// epoch sequence, so any protocol mix keeps "flag >= target" meaningful.
+enum : uint64_t { kPhaseTop = 1, kPhaseMid = 2, kPhaseBottom = 3 };
+
+// LL128 geometry: a line is 120 data bytes (60 bf16) + an 8-byte flag word;
+// a warp moves 4 lines (8 lanes x 16 bytes each) per step.
+constexpr int kLL128Elems = 60;
+constexpr int kLL128Line = 128;
+constexpr int kLL128LinesPerWarp = 4;
+
+// LL geometry: one 16-byte input vector (8 bf16) becomes four 8-byte units
+// (2 bf16 + 32-bit epoch each), written as two 16-byte stores. The two halves
+// of 32 consecutive vectors are laid out lane-interleaved (512 + 512 bytes)
+// so that each warp-wide store covers whole 32-byte sectors.
+constexpr int kLLChunkVecs = 32;
+constexpr int kLLChunkBytes = 1024;
+
+// Device status block (one per context).
+struct DevStatus {
+  int code;       // first sfc_status error recorded (0 = none)
+  uint32_t info;  // detail: (op << 16) | (rank << 8) | source
+  int abort;      // nonzero: every wait and every later kernel exits
+  int pad;
+};
+
+// Kernel parameters (passed by value as a __grid_constant__).
+struct KParams {
+  // operand addressing: mode 0 = inline pointers (one operation),
+  // 1 = device pointer tables [k * N + r], 2 = strided from a base.
+  const uint16_t* in_inline[kMaxRanks];
+  uint16_t* out_inline[kMaxRanks];
+  const uint16_t* const* in_table;
+  uint16_t* const* out_table;
+  const uint16_t* in_base;
+  uint16_t* out_base;
+  uint64_t in_stride;   // elements between consecutive (k, r) inputs
+  uint64_t out_stride;  // elements between consecutive (k, r) outputs
+  int addr_mode;
+
+  uint64_t count;       // elements per rank (all-gather: per shard)
+  int k_ops;            // operations in this launch
+  int G;                // CTAs per rank
+  uint32_t first_epoch;
+
+  uint8_t* scratch;     // protocol region; slot (recv, parity, j) at
+                        // ((recv * 2 + parity) * (N - 1) + j) * slot_stride
+  uint64_t slot_stride; // bytes
+  uint64_t* bar;        // barrier counters [N][bar_stride]
+  int bar_stride;
+  uint16_t* red;        // twoshot reduced shards [N][red_stride]
+  uint64_t red_stride;  // elements
+
+  DevStatus* status;
+  uint64_t* timings;    // [k_ops + 1] or null
+  const uint32_t* skew; // [k_ops * N] ns or null
+  uint64_t timeout_ns;
+  int debug;
+  int silent_rank;      // -1 = none
+};
+
+// Kernel entry for (nranks, protocol, op); null if not provided.
+const void* kernel_for(int nranks, int protocol, int op);
+
+// Encoded slot size (bytes) for `count` elements under the GPU layout.
+uint64_t slot_bytes_gpu(int protocol, uint64_t count);
+
+}  // namespace sfc

@@ -1,0 +1,531 @@
+// Persistent collective kernels: N emulated ranks, G CTAs per rank, k_ops
+// operations per launch.
+//
+// Rank r owns CTAs [r * G, (r + 1) * G). Every operation uses the same
+// element -> (CTA, thread) mapping, so thread t of CTA k of every rank forms
+// an independent self-synchronizing pipeline: it pushes its elements of
+// operation e, then polls the same elements from every peer, and the peers'
+// threads with the same index do the same. A writer reaches epoch e+2 only
+// after the reader's epoch e+1 push arrived, which the reader issues only
+// after it consumed epoch e (and, for the sentinel, rewrote the slot); a
+// fence.acq_rel.gpu between the end of one operation and the pushes of the
+// next makes that ordering hold in the memory model. That is the double
+// buffering of "Why Microseconds Matter in AI Infrastructure", section
+// "Latency can matter more than bandwidth": receipt of data is the evidence
+// that the other buffer can be reused, with no global barrier.
+//
+// Within an operation a warp polls all its sources at once (independent
+// loads, one round trip per poll) and the warp decides with a vote whether
+// to poll again, so lanes never diverge in the wait loop. Sources are taken
+// in arrival order; the reduction runs in rank order 0..N-1 on registers
+// ("flash-comm: Self-Synchronizing Collective Communication for LLM
+// Decoding", abstract: transport order decoupled from reduction order).
+#include <cuda_runtime.h>
+
+#include "sfc_device.cuh"
+
+namespace sfc {
+
+// ---------------------------------------------------------------- addressing
+template <int N>
+SFC_DEV const uint16_t* in_ptr(const KParams& p, int op, int r) {
+  if (p.addr_mode == 0) return p.in_inline[r];
+  if (p.addr_mode == 1) return ld_nc_ptr(&p.in_table[op * N + r]);
+  return p.in_base + (static_cast<uint64_t>(op) * N + r) * p.in_stride;
+}
+template <int N>
+SFC_DEV uint16_t* out_ptr(const KParams& p, int op, int r) {
+  if (p.addr_mode == 0) return p.out_inline[r];
+  if (p.addr_mode == 1) return ld_nc_ptr(&p.out_table[op * N + r]);
+  return p.out_base + (static_cast<uint64_t>(op) * N + r) * p.out_stride;
+}
+// Receive slot of `recv` for data from `src` (src != recv) at `par`.
+template <int N>
+SFC_DEV uint8_t* slot_ptr(const KParams& p, int recv, int par, int src) {
+  const int j = src < recv ? src : src - 1;
+  return p.scratch + static_cast<uint64_t>((recv * 2 + par) * (N - 1) + j) * p.slot_stride;
+}
+
+SFC_DEV uint64_t ll_off(uint64_t v, int half) {
+  return ((v >> 5) << 10) + (static_cast<uint64_t>(half) << 9) + ((v & 31) << 4);
+}
+
+// One deferred output vector: the last result of an operation is written
+// after the next operation's pushes, so the per-operation fence does not wait
+// for its store to be acknowledged.
+struct PendingOut {
+  uint16_t* base = nullptr;
+  uint64_t e0 = 0, limit = 0;
+  uint4 v = make_uint4(0, 0, 0, 0);
+  bool valid = false;
+  SFC_DEV void flush() {
+    if (valid) store_n(base, e0, v, 8, limit);
+    valid = false;
+  }
+  SFC_DEV void set(uint16_t* b, uint64_t e, uint4 x, uint64_t lim) {
+    flush();
+    base = b;
+    e0 = e;
+    v = x;
+    limit = lim;
+    valid = true;
+  }
+};
+
+// ===================================================================== LL
+// Unit = 8 bytes {2 bf16, epoch}; a 16-byte input vector v becomes units
+// 4v..4v+3 stored as two .v2.b64 stores. Readiness: all four epoch words of
+// the two loads equal e.
+template <int N, int OP>
+SFC_DEV bool ll_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid, uint64_t gstride,
+                   PendingOut& pend) {
+  const uint64_t count = p.count;
+  const uint64_t nvec = (count + 7) >> 3;
+  const int par = e & 1;
+  const uint64_t ehi = static_cast<uint64_t>(e) << 32;
+  const int lane = threadIdx.x & 31;
+  const uint16_t* in_r = in_ptr<N>(p, op, r);
+  uint16_t* out_r = out_ptr<N>(p, op, r);
+
+  if (r != p.silent_rank) {
+    for (uint64_t v = gtid; v < nvec; v += gstride) {
+      const uint4 x = load8(in_r, v * 8, count);
+      const uint64_t o0 = ll_off(v, 0), o1 = ll_off(v, 1);
+#pragma unroll
+      for (int q = 0; q < N; ++q) {
+        if (q == r) continue;
+        uint8_t* s = slot_ptr<N>(p, q, par, r);
+        st_rlx_v2u64(s + o0, ehi | x.x, ehi | x.y);
+        st_rlx_v2u64(s + o1, ehi | x.z, ehi | x.w);
+      }
+    }
+  }
+  pend.flush();
+
+  const uint8_t* my = slot_ptr<N>(p, r, par, r == 0 ? 1 : 0);  // slot j = 0
+  for (uint64_t vb = gtid - lane; vb < nvec; vb += gstride) {
+    const uint64_t v = vb + lane;
+    const bool act = v < nvec;
+    uint4 x[N];
+    const uint4 own = act ? load8(in_r, v * 8, count) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int q = 0; q < N; ++q) x[q] = own;
+    uint32_t need = act ? (((1u << N) - 1u) & ~(1u << r)) : 0u;
+    const uint64_t o0 = ll_off(v, 0), o1 = ll_off(v, 1);
+    WarpWait ww;
+    while (true) {
+#pragma unroll
+      for (int q = 0; q < N; ++q) {
+        if (need & (1u << q)) {
+          const int j = q < r ? q : q - 1;
+          const uint8_t* s = my + static_cast<uint64_t>(j) * p.slot_stride;
+          uint64_t a, b, c, d;
+          ld_rlx_v2u64(s + o0, a, b);
+          ld_rlx_v2u64(s + o1, c, d);
+          const bool ok = static_cast<uint32_t>(a >> 32) == e && static_cast<uint32_t>(b >> 32) == e &&
+                          static_cast<uint32_t>(c >> 32) == e && static_cast<uint32_t>(d >> 32) == e;
+          if (ok) {
+            x[q] = make_uint4(static_cast<uint32_t>(a), static_cast<uint32_t>(b), static_cast<uint32_t>(c),
+                              static_cast<uint32_t>(d));
+            need &= ~(1u << q);
+          }
+        }
+      }
+      if (!__any_sync(kFull, need != 0u)) break;
+      if (ww.tick(p, op, r, need ? __ffs(need) - 1 : -1)) return false;
+    }
+    if (act) {
+      if (OP == kAllreduce) {
+        pend.set(out_r, v * 8, reduce8<N>(x), count);
+      } else {
+#pragma unroll
+        for (int q = 0; q < N; ++q) store_n(out_r, q * count + v * 8, x[q], 8, q * count + count);
+      }
+    }
+  }
+  return true;
+}
+
+// ================================================================ sentinel
+// Raw 16-byte vectors into a slot pre-filled with 0xFFFF; a vector is ready
+// when none of its 8 elements is 0xFFFF; after consuming, the reader writes
+// 0xFFFF back before its next push (ordered by the per-operation fence).
+template <int N, int OP>
+SFC_DEV bool sentinel_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid, uint64_t gstride,
+                         PendingOut& pend) {
+  const uint64_t count = p.count;
+  const uint64_t nvec = (count + 7) >> 3;
+  const int par = e & 1;
+  const int lane = threadIdx.x & 31;
+  const uint16_t* in_r = in_ptr<N>(p, op, r);
+  uint16_t* out_r = out_ptr<N>(p, op, r);
+
+  if (r != p.silent_rank) {
+    for (uint64_t v = gtid; v < nvec; v += gstride) {
+      const uint4 x = load8(in_r, v * 8, count);
+      // the receivers of a sentinel element would never see it arrive: record
+      // the error; every wait then sees the abort word and exits
+      if (p.debug && has_sentinel(x)) record_error(p, 6 /* SFC_ERR_SENTINEL_IN_INPUT */, err_info(op, r, r));
+#pragma unroll
+      for (int q = 0; q < N; ++q) {
+        if (q == r) continue;
+        st_rlx_v4u32(slot_ptr<N>(p, q, par, r) + v * 16, x);
+      }
+    }
+  }
+  pend.flush();
+
+  const uint8_t* my = slot_ptr<N>(p, r, par, r == 0 ? 1 : 0);
+  const uint4 fill = make_uint4(kFull, kFull, kFull, kFull);
+  for (uint64_t vb = gtid - lane; vb < nvec; vb += gstride) {
+    const uint64_t v = vb + lane;
+    const bool act = v < nvec;
+    uint4 x[N];
+    const uint4 own = act ? load8(in_r, v * 8, count) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int q = 0; q < N; ++q) x[q] = own;
+    uint32_t need = act ? (((1u << N) - 1u) & ~(1u << r)) : 0u;
+    WarpWait ww;
+    while (true) {
+#pragma unroll
+      for (int q = 0; q < N; ++q) {
+        if (need & (1u << q)) {
+          const int j = q < r ? q : q - 1;
+          const uint4 y = ld_rlx_v4u32(my + static_cast<uint64_t>(j) * p.slot_stride + v * 16);
+          if (!has_sentinel(y)) {
+            x[q] = y;
+            need &= ~(1u << q);
+          }
+        }
+      }
+      if (!__any_sync(kFull, need != 0u)) break;
+      if (ww.tick(p, op, r, need ? __ffs(need) - 1 : -1)) return false;
+    }
+    if (act) {
+#pragma unroll
+      for (int j = 0; j < N - 1; ++j) st_rlx_v4u32(const_cast<uint8_t*>(my) + j * p.slot_stride + v * 16, fill);
+      if (OP == kAllreduce) {
+        pend.set(out_r, v * 8, reduce8<N>(x), count);
+      } else {
+#pragma unroll
+        for (int q = 0; q < N; ++q) store_n(out_r, q * count + v * 8, x[q], 8, q * count + count);
+      }
+    }
+  }
+  return true;
+}
+
+// =================================================================== LL128
+// A line = 120 data bytes (60 bf16) + 8-byte flag (= epoch). A warp moves 4
+// lines: lane l serves line 4g + (l >> 3), sub-slot s = l & 7; lanes s < 7
+// carry 16 data bytes at line offset 16 s, lane 7 carries the last 8 data
+// bytes (offset 112) and the flag (offset 120). Writers store all data,
+// __syncwarp + fence.acq_rel.gpu, then the flags (release pattern); readers
+// poll flags with relaxed loads, fence.acq_rel.gpu + __syncwarp (acquire
+// pattern), then load the data. Flags of up to B line groups are polled at
+// once.
+template <int N>
+struct LL128Batch {
+  static constexpr int B = 32 / N;  // bits b * N + q of one 32-bit mask
+};
+
+template <int N, int OP>
+SFC_DEV bool ll128_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid, uint64_t gstride) {
+  constexpr int B = LL128Batch<N>::B;
+  const uint64_t count = p.count;
+  const uint64_t nlines = (count + kLL128Elems - 1) / kLL128Elems;
+  const uint64_t ngroups = (nlines + kLL128LinesPerWarp - 1) / kLL128LinesPerWarp;
+  const int par = e & 1;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane & 7;
+  const uint64_t lsel = static_cast<uint64_t>(lane >> 3);
+  const uint64_t wg = gtid >> 5, wstride = gstride >> 5;
+  const uint16_t* in_r = in_ptr<N>(p, op, r);
+  uint16_t* out_r = out_ptr<N>(p, op, r);
+  const uint32_t peers = ((1u << N) - 1u) & ~(1u << r);
+
+  if (r != p.silent_rank) {
+    for (uint64_t g = wg; g < ngroups; g += wstride) {
+      const uint64_t L = g * kLL128LinesPerWarp + lsel;
+      if (L < nlines) {
+        const uint64_t e0 = L * kLL128Elems + sub * 8;
+        const uint2 lo = load4(in_r, e0, count);
+        const uint2 hi = sub < 7 ? load4(in_r, e0 + 4, count) : make_uint2(0u, 0u);
+#pragma unroll
+        for (int q = 0; q < N; ++q) {
+          if (q == r) continue;
+          uint8_t* s = slot_ptr<N>(p, q, par, r) + L * kLL128Line + sub * 16;
+          if (sub < 7)
+            st_rlx_v4u32(s, make_uint4(lo.x, lo.y, hi.x, hi.y));
+          else
+            st_rlx_v2u32(s, lo);
+        }
+      }
+    }
+    __syncwarp();
+    fence_acq_rel();
+    for (uint64_t g = wg; g < ngroups; g += wstride) {
+      const uint64_t L = g * kLL128LinesPerWarp + lsel;
+      if (L < nlines && sub == 7) {
+#pragma unroll
+        for (int q = 0; q < N; ++q) {
+          if (q == r) continue;
+          st_rlx_u64(slot_ptr<N>(p, q, par, r) + L * kLL128Line + 120, static_cast<uint64_t>(e));
+        }
+      }
+    }
+  }
+
+  const uint8_t* my = slot_ptr<N>(p, r, par, r == 0 ? 1 : 0);
+  for (uint64_t g0 = wg; g0 < ngroups; g0 += wstride * B) {
+    uint32_t need = 0;
+    if (sub == 7) {
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        const uint64_t g = g0 + b * wstride;
+        const uint64_t L = g * kLL128LinesPerWarp + lsel;
+        if (g < ngroups && L < nlines) need |= peers << (b * N);
+      }
+    }
+    WarpWait ww;
+    while (true) {
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        const uint64_t L = (g0 + b * wstride) * kLL128LinesPerWarp + lsel;
+#pragma unroll
+        for (int q = 0; q < N; ++q) {
+          if (need & (1u << (b * N + q))) {
+            const int j = q < r ? q : q - 1;
+            const uint64_t f = ld_rlx_u64(my + static_cast<uint64_t>(j) * p.slot_stride + L * kLL128Line + 120);
+            if (f == static_cast<uint64_t>(e)) need &= ~(1u << (b * N + q));
+          }
+        }
+      }
+      if (!__any_sync(kFull, need != 0u)) break;
+      if (ww.tick(p, op, r, -1)) return false;
+    }
+    fence_acq_rel();
+    __syncwarp();
+#pragma unroll 1
+    for (int b = 0; b < B; ++b) {
+      const uint64_t g = g0 + b * wstride;
+      const uint64_t L = g * kLL128LinesPerWarp + lsel;
+      if (g >= ngroups || L >= nlines) continue;
+      const uint64_t e0 = L * kLL128Elems + sub * 8;
+      const int n = sub < 7 ? 8 : 4;
+      const uint2 olo = load4(in_r, e0, count);
+      const uint2 ohi = sub < 7 ? load4(in_r, e0 + 4, count) : make_uint2(0u, 0u);
+      const uint4 own = make_uint4(olo.x, olo.y, ohi.x, ohi.y);
+      uint4 x[N];
+#pragma unroll
+      for (int q = 0; q < N; ++q) {
+        if (q == r) {
+          x[q] = own;
+        } else {
+          const int j = q < r ? q : q - 1;
+          const uint8_t* s = my + static_cast<uint64_t>(j) * p.slot_stride + L * kLL128Line + sub * 16;
+          if (sub < 7) {
+            x[q] = ld_rlx_v4u32(s);
+          } else {
+            const uint2 t = ld_rlx_v2u32(s);
+            x[q] = make_uint4(t.x, t.y, 0u, 0u);
+          }
+        }
+      }
+      if (OP == kAllreduce) {
+        store_n(out_r, e0, reduce8<N>(x), n, count);
+      } else {
+#pragma unroll
+        for (int q = 0; q < N; ++q) store_n(out_r, q * count + e0, x[q], n, q * count + count);
+      }
+    }
+  }
+  return true;
+}
+
+// ============================================================ barriers
+// Per-CTA-index barrier: CTA k of rank r publishes (epoch << 2) | phase with
+// a release store and waits until CTA k of every rank has published at least
+// that (acquire loads by threads 0..N-1). CTA-uniform result.
+template <int N>
+SFC_DEV bool cta_barrier(const KParams& p, int r, int k, int op, uint64_t target) {
+  __syncthreads();
+  int bad = 0;
+  if (threadIdx.x == 0 && r != p.silent_rank)
+    st_rel_u64(&p.bar[static_cast<uint64_t>(r) * p.bar_stride + k], target);
+  if (threadIdx.x < N) {
+    const uint64_t* f = &p.bar[static_cast<uint64_t>(threadIdx.x) * p.bar_stride + k];
+    ThreadWait tw;
+    while (ld_acq_u64(f) < target) {
+      if (tw.tick(p, op, r, threadIdx.x)) {
+        bad = 1;
+        break;
+      }
+    }
+  }
+  return __syncthreads_or(bad) == 0;
+}
+
+// Oneshot (pull): top barrier, read every rank's input, reduce in rank
+// order (all-gather: copy), bottom barrier ("SiFAR: Synchronization-Free
+// All-Reduce for Low-Latency LLM Inference", abstract).
+template <int N, int OP>
+SFC_DEV bool oneshot_op(const KParams& p, int r, int k, int op, uint32_t e, uint64_t gtid, uint64_t gstride) {
+  const uint64_t count = p.count;
+  const uint64_t nvec = (count + 7) >> 3;
+  const uint64_t eb = static_cast<uint64_t>(e) << 2;
+  if (!cta_barrier<N>(p, r, k, op, eb | kPhaseTop)) return false;
+  uint16_t* out_r = out_ptr<N>(p, op, r);
+  const uint16_t* src[N];
+#pragma unroll
+  for (int q = 0; q < N; ++q) src[q] = in_ptr<N>(p, op, q);
+  for (uint64_t v = gtid; v < nvec; v += gstride) {
+    uint4 x[N];
+#pragma unroll
+    for (int q = 0; q < N; ++q) x[q] = load8(src[q], v * 8, count);
+    if (OP == kAllreduce) {
+      store_n(out_r, v * 8, reduce8<N>(x), 8, count);
+    } else {
+#pragma unroll
+      for (int q = 0; q < N; ++q) store_n(out_r, q * count + v * 8, x[q], 8, q * count + count);
+    }
+  }
+  return cta_barrier<N>(p, r, k, op, eb | kPhaseBottom);
+}
+
+// Twoshot (pull): top barrier; reduce-scatter (rank r reduces shard r of
+// every input into its reduction buffer and its output); middle barrier;
+// all-gather (copy every other rank's reduced shard); bottom barrier. CTA k
+// of each rank covers the same vector offsets inside every shard, so the
+// per-CTA-index barriers order each producer before its consumers.
+template <int N>
+SFC_DEV bool twoshot_op(const KParams& p, int r, int k, int op, uint32_t e, uint64_t gtid, uint64_t gstride) {
+  const uint64_t count = p.count;
+  const uint64_t nvec = (count + 7) >> 3;
+  const uint64_t sv = (nvec + N - 1) / N;  // vectors per shard
+  const uint64_t eb = static_cast<uint64_t>(e) << 2;
+  if (!cta_barrier<N>(p, r, k, op, eb | kPhaseTop)) return false;
+  uint16_t* out_r = out_ptr<N>(p, op, r);
+  {
+    const uint16_t* src[N];
+#pragma unroll
+    for (int q = 0; q < N; ++q) src[q] = in_ptr<N>(p, op, q);
+    const uint64_t lo = r * sv, hi = min(lo + sv, nvec);
+    uint16_t* red = p.red + static_cast<uint64_t>(r) * p.red_stride;
+    for (uint64_t v = lo + gtid; v < hi; v += gstride) {
+      uint4 x[N];
+#pragma unroll
+      for (int q = 0; q < N; ++q) x[q] = load8(src[q], v * 8, count);
+      const uint4 y = reduce8<N>(x);
+      *reinterpret_cast<uint4*>(red + (v - lo) * 8) = y;
+      store_n(out_r, v * 8, y, 8, count);
+    }
+  }
+  if (!cta_barrier<N>(p, r, k, op, eb | kPhaseMid)) return false;
+#pragma unroll 1
+  for (int q = 0; q < N; ++q) {
+    if (q == r) continue;
+    const uint64_t lo = q * sv, hi = min(lo + sv, nvec);
+    const uint16_t* red = p.red + static_cast<uint64_t>(q) * p.red_stride;
+    for (uint64_t v = lo + gtid; v < hi; v += gstride) {
+      const uint4 y = ld_rlx_v4u32(red + (v - lo) * 8);
+      store_n(out_r, v * 8, y, 8, count);
+    }
+  }
+  return cta_barrier<N>(p, r, k, op, eb | kPhaseBottom);
+}
+
+// ============================================================== the kernel
+template <int N, int PROTO, int OP>
+__global__ void __launch_bounds__(kThreads, 2) sfc_kernel(const __grid_constant__ KParams p) {
+  const int r = blockIdx.x / p.G;
+  const int k = blockIdx.x - r * p.G;
+  const uint64_t gtid = static_cast<uint64_t>(k) * kThreads + threadIdx.x;
+  const uint64_t gstride = static_cast<uint64_t>(p.G) * kThreads;
+  const int lane = threadIdx.x & 31;
+  if (ld_rlx_s32(&p.status->abort)) return;  // poisoned context: do nothing
+  if (p.timings != nullptr && lane == 0)
+    atomicMin(reinterpret_cast<unsigned long long*>(&p.timings[0]), static_cast<unsigned long long>(gtimer()));
+  PendingOut pend;
+  for (int op = 0; op < p.k_ops; ++op) {
+    const uint32_t e = p.first_epoch + static_cast<uint32_t>(op);
+    if (PROTO == kLL || PROTO == kLL128 || PROTO == kSentinel) {
+      // end of the previous operation's reads / resets before these pushes
+      if (op > 0) fence_acq_rel();
+    }
+    if (p.skew != nullptr) spin_ns(__ldg(&p.skew[op * N + r]), p.timeout_ns);
+    bool ok;
+    if (PROTO == kLL)
+      ok = ll_op<N, OP>(p, r, op, e, gtid, gstride, pend);
+    else if (PROTO == kSentinel)
+      ok = sentinel_op<N, OP>(p, r, op, e, gtid, gstride, pend);
+    else if (PROTO == kLL128)
+      ok = ll128_op<N, OP>(p, r, op, e, gtid, gstride);
+    else if (PROTO == kOneshot)
+      ok = oneshot_op<N, OP>(p, r, k, op, e, gtid, gstride);
+    else
+      ok = twoshot_op<N>(p, r, k, op, e, gtid, gstride);
+    if (!ok) return;
+    if (p.timings != nullptr && lane == 0)
+      atomicMax(reinterpret_cast<unsigned long long*>(&p.timings[1 + op]), static_cast<unsigned long long>(gtimer()));
+  }
+  pend.flush();
+}
+
+// ============================================================ dispatch table
+namespace {
+template <int N>
+struct Row {
+  static void fill(const void* (&t)[kMaxRanks + 1][6][2]) {
+    t[N][kLL][kAllreduce] = reinterpret_cast<const void*>(&sfc_kernel<N, kLL, kAllreduce>);
+    t[N][kLL][kAllgather] = reinterpret_cast<const void*>(&sfc_kernel<N, kLL, kAllgather>);
+    t[N][kLL128][kAllreduce] = reinterpret_cast<const void*>(&sfc_kernel<N, kLL128, kAllreduce>);
+    t[N][kLL128][kAllgather] = reinterpret_cast<const void*>(&sfc_kernel<N, kLL128, kAllgather>);
+    t[N][kSentinel][kAllreduce] = reinterpret_cast<const void*>(&sfc_kernel<N, kSentinel, kAllreduce>);
+    t[N][kSentinel][kAllgather] = reinterpret_cast<const void*>(&sfc_kernel<N, kSentinel, kAllgather>);
+    t[N][kOneshot][kAllreduce] = reinterpret_cast<const void*>(&sfc_kernel<N, kOneshot, kAllreduce>);
+    t[N][kOneshot][kAllgather] = reinterpret_cast<const void*>(&sfc_kernel<N, kOneshot, kAllgather>);
+    t[N][kTwoshot][kAllreduce] = reinterpret_cast<const void*>(&sfc_kernel<N, kTwoshot, kAllreduce>);
+    t[N][kTwoshot][kAllgather] = nullptr;
+  }
+};
+
+struct Table {
+  const void* t[kMaxRanks + 1][6][2] = {};
+  Table() {
+    Row<2>::fill(t);
+    Row<3>::fill(t);
+    Row<4>::fill(t);
+    Row<5>::fill(t);
+    Row<6>::fill(t);
+    Row<7>::fill(t);
+    Row<8>::fill(t);
+  }
+};
+}  // namespace
+
+const void* kernel_for(int nranks, int protocol, int op) {
+  static const Table table;
+  if (nranks < kMinRanks || nranks > kMaxRanks || protocol < kLL || protocol > kTwoshot || op < 0 || op > 1)
+    return nullptr;
+  return table.t[nranks][protocol][op];
+}
+
+uint64_t slot_bytes_gpu(int protocol, uint64_t count) {
+  const uint64_t nvec = (count + 7) / 8;
+  switch (protocol) {
+    case kLL:
+      return ((nvec + kLLChunkVecs - 1) / kLLChunkVecs) * kLLChunkBytes;
+    case kLL128: {
+      const uint64_t lines = (count + kLL128Elems - 1) / kLL128Elems;
+      const uint64_t groups = (lines + kLL128LinesPerWarp - 1) / kLL128LinesPerWarp;
+      return groups * kLL128LinesPerWarp * kLL128Line;
+    }
+    case kSentinel:
+      return nvec * 16;
+    default:
+      return 0;
+  }
+}
+
+}  // namespace sfc

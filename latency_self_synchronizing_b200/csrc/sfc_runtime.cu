@@ -1,0 +1,539 @@
+// Host runtime of libsfc: context, argument checks, epoch sequence, scratch
+// provisioning, launch shape, cooperative launch, status, selector.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "sfc.h"
+#include "sfc_internal.h"
+
+using namespace sfc;
+
+struct sfc_ctx {
+  int device = 0;
+  int nranks = 0;
+  size_t max_bytes = 0;
+  uint64_t max_count = 0;
+  sfc_config cfg{};
+  int sm_count = 0;
+
+  uint8_t* region[6] = {};     // per self-sync protocol scratch
+  uint64_t slot_stride[6] = {};
+  uint64_t region_bytes[6] = {};
+  uint64_t* bar = nullptr;
+  int bar_stride = 0;
+  uint16_t* red = nullptr;
+  uint64_t red_stride = 0;
+  DevStatus* dstatus = nullptr;
+  DevStatus* hstatus = nullptr;  // page-locked mirror
+
+  uint32_t next_epoch = 1;
+  bool poisoned = false;
+  int silent_rank = -1;
+  cudaStream_t last_stream = nullptr;
+  uint64_t launches = 0;
+  sfc_cost_model model{};
+
+  int occupancy[6][2] = {};  // blocks per SM, per (protocol, op), 0 = unknown
+
+  // staging for the host-buffer entry point
+  uint16_t* stage_in = nullptr;
+  uint16_t* stage_out = nullptr;
+  size_t stage_bytes = 0;
+};
+
+namespace {
+
+constexpr uint32_t kDefaultTimeoutUs = 50000;
+constexpr int kBarStride = 1024;  // >= any CTAs-per-rank value
+
+bool cuda_ok(cudaError_t e) {
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  return true;
+}
+
+bool self_sync(int proto) { return proto == kLL || proto == kLL128 || proto == kSentinel; }
+
+bool provisioned(const sfc_ctx* c, int proto) {
+  const uint32_t mask = c->cfg.protocol_mask ? c->cfg.protocol_mask : 0x3Eu;
+  return (mask >> proto) & 1u;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// [a, a + n) and [b, b + m) overlap?
+bool overlap(const void* a, size_t n, const void* b, size_t m) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + m && y < x + n;
+}
+
+int occupancy_of(sfc_ctx* c, int proto, int op) {
+  int& occ = c->occupancy[proto][op];
+  if (occ == 0) {
+    const void* fn = kernel_for(c->nranks, proto, op);
+    int nb = 0;
+    if (fn == nullptr || !cuda_ok(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, kThreads, 0)))
+      return 0;
+    occ = nb;
+  }
+  return occ;
+}
+
+// CTAs per rank for a call: enough threads for one unit of work each
+// (an 8-element vector, or a 4-line LL128 group per warp), capped so that
+// all N * G CTAs are co-resident.
+int choose_G(sfc_ctx* c, int proto, int op, uint64_t count, int* gmax_out) {
+  const int occ = occupancy_of(c, proto, op);
+  const int gmax = std::min(kBarStride, occ * c->sm_count / c->nranks);
+  if (gmax_out) *gmax_out = gmax;
+  if (gmax <= 0) return 0;
+  if (c->cfg.ctas_per_rank > 0) return c->cfg.ctas_per_rank;
+  const uint64_t nvec = (count + 7) / 8;
+  uint64_t threads_needed;
+  if (proto == kLL128) {
+    const uint64_t lines = (count + kLL128Elems - 1) / kLL128Elems;
+    threads_needed = (lines + kLL128LinesPerWarp - 1) / kLL128LinesPerWarp * 32;
+  } else if (proto == kTwoshot) {
+    threads_needed = (nvec + c->nranks - 1) / c->nranks;
+  } else {
+    threads_needed = nvec;
+  }
+  uint64_t g = (threads_needed + kThreads - 1) / kThreads;
+  g = std::max<uint64_t>(1, std::min<uint64_t>(g, gmax));
+  return static_cast<int>(g);
+}
+
+sfc_status check_common(sfc_ctx* c, sfc_op op, size_t count, sfc_dtype dtype, int proto, uint32_t first_epoch,
+                        int k_ops) {
+  if (c == nullptr || k_ops < 1) return SFC_ERR_INVALID;
+  if (dtype != SFC_BF16) return SFC_ERR_UNSUPPORTED;
+  if (op != SFC_OP_ALLREDUCE && op != SFC_OP_ALLGATHER) return SFC_ERR_INVALID;
+  if (proto < kLL || proto > kTwoshot) return SFC_ERR_INVALID;
+  if (op == SFC_OP_ALLGATHER && proto == kTwoshot) return SFC_ERR_UNSUPPORTED;
+  if (!provisioned(c, proto)) return SFC_ERR_UNSUPPORTED;
+  if (count > c->max_count) return SFC_ERR_INVALID;
+  if (c->poisoned) return SFC_ERR_ABORTED;
+  if (first_epoch != c->next_epoch) return SFC_ERR_EPOCH;
+  if (static_cast<uint64_t>(first_epoch) + static_cast<uint64_t>(k_ops) - 1 > 0xFFFFFFFFull) return SFC_ERR_EPOCH;
+  return SFC_OK;
+}
+
+void fill_common(sfc_ctx* c, KParams& p, int proto, uint64_t count, int k_ops, uint32_t first_epoch, int G) {
+  p.count = count;
+  p.k_ops = k_ops;
+  p.G = G;
+  p.first_epoch = first_epoch;
+  p.scratch = self_sync(proto) ? c->region[proto] : nullptr;
+  p.slot_stride = self_sync(proto) ? c->slot_stride[proto] : 0;
+  p.bar = c->bar;
+  p.bar_stride = c->bar_stride;
+  p.red = c->red;
+  p.red_stride = c->red_stride;
+  p.status = c->dstatus;
+  p.timeout_ns = static_cast<uint64_t>(c->cfg.timeout_us ? c->cfg.timeout_us : kDefaultTimeoutUs) * 1000ull;
+  p.debug = c->cfg.debug_checks;
+  p.silent_rank = c->silent_rank;
+}
+
+sfc_status launch(sfc_ctx* c, int proto, int op, KParams& p, cudaStream_t stream) {
+  const void* fn = kernel_for(c->nranks, proto, op);
+  if (fn == nullptr) return SFC_ERR_UNSUPPORTED;
+  int gmax = 0;
+  (void)choose_G(c, proto, op, p.count, &gmax);
+  if (p.G < 1 || p.G > gmax) return SFC_ERR_RESOURCES;
+  void* args[] = {&p};
+  cudaError_t e = cudaLaunchCooperativeKernel(fn, dim3(c->nranks * p.G), dim3(kThreads), args, 0, stream);
+  if (e == cudaErrorCooperativeLaunchTooLarge) {
+    (void)cudaGetLastError();
+    return SFC_ERR_RESOURCES;
+  }
+  if (!cuda_ok(e)) return SFC_ERR_CUDA;
+  c->launches++;
+  c->last_stream = stream;
+  return SFC_OK;
+}
+
+sfc_status prepare_timings(uint64_t* timings, int k_ops, cudaStream_t stream) {
+  if (timings == nullptr) return SFC_OK;
+  if (!cuda_ok(cudaMemsetAsync(timings, 0xFF, sizeof(uint64_t), stream))) return SFC_ERR_CUDA;
+  if (!cuda_ok(cudaMemsetAsync(timings + 1, 0, sizeof(uint64_t) * k_ops, stream))) return SFC_ERR_CUDA;
+  return SFC_OK;
+}
+
+sfc_status one_op(sfc_ctx* c, sfc_op op, const void* const* in, void* const* out, size_t count, sfc_dtype dtype,
+                  sfc_protocol protocol, uint32_t epoch, void* stream) {
+  if (c == nullptr || in == nullptr || out == nullptr) return SFC_ERR_INVALID;
+  if (count == 0) return (dtype == SFC_BF16) ? SFC_OK : SFC_ERR_UNSUPPORTED;
+  int proto = protocol;
+  if (proto == SFC_PROTO_AUTO) proto = sfc_select_protocol(c, op, count * 2, c->nranks);
+  sfc_status s = check_common(c, op, count, dtype, proto, epoch, 1);
+  if (s != SFC_OK) return s;
+  const int N = c->nranks;
+  const size_t in_bytes = count * 2;
+  const size_t out_bytes = (op == SFC_OP_ALLGATHER ? N : 1) * count * 2;
+  for (int r = 0; r < N; ++r) {
+    if (in[r] == nullptr || out[r] == nullptr || !aligned16(in[r]) || !aligned16(out[r])) return SFC_ERR_INVALID;
+  }
+  for (int a = 0; a < N; ++a) {
+    for (int b = 0; b < N; ++b) {
+      if (overlap(in[a], in_bytes, out[b], out_bytes)) return SFC_ERR_INVALID;
+      if (a < b && overlap(out[a], out_bytes, out[b], out_bytes)) return SFC_ERR_INVALID;
+    }
+  }
+  KParams p{};
+  for (int r = 0; r < N; ++r) {
+    p.in_inline[r] = static_cast<const uint16_t*>(in[r]);
+    p.out_inline[r] = static_cast<uint16_t*>(out[r]);
+  }
+  p.addr_mode = 0;
+  const int G = choose_G(c, proto, op, count, nullptr);
+  fill_common(c, p, proto, count, 1, epoch, G);
+  s = launch(c, proto, op, p, static_cast<cudaStream_t>(stream));
+  if (s == SFC_OK) c->next_epoch = epoch + 1;
+  return s;
+}
+
+sfc_status chain(sfc_ctx* c, sfc_op op, int k_ops, const void* const* in_table, void* const* out_table, size_t count,
+                 sfc_dtype dtype, sfc_protocol protocol, uint32_t first_epoch, const uint32_t* skew_ns,
+                 uint64_t* timings, void* stream) {
+  if (c == nullptr || in_table == nullptr || out_table == nullptr) return SFC_ERR_INVALID;
+  if (count == 0) return (dtype == SFC_BF16 && k_ops >= 1) ? SFC_OK : SFC_ERR_INVALID;
+  int proto = protocol;
+  if (proto == SFC_PROTO_AUTO) proto = sfc_select_protocol(c, op, count * 2, c->nranks);
+  sfc_status s = check_common(c, op, count, dtype, proto, first_epoch, k_ops);
+  if (s != SFC_OK) return s;
+  if ((reinterpret_cast<uintptr_t>(in_table) | reinterpret_cast<uintptr_t>(out_table)) & 7u) return SFC_ERR_INVALID;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = prepare_timings(timings, k_ops, st);
+  if (s != SFC_OK) return s;
+  KParams p{};
+  p.addr_mode = 1;
+  p.in_table = reinterpret_cast<const uint16_t* const*>(in_table);
+  p.out_table = reinterpret_cast<uint16_t* const*>(out_table);
+  p.skew = skew_ns;
+  p.timings = timings;
+  const int G = choose_G(c, proto, op, count, nullptr);
+  fill_common(c, p, proto, count, k_ops, first_epoch, G);
+  s = launch(c, proto, op, p, st);
+  if (s == SFC_OK) c->next_epoch = first_epoch + static_cast<uint32_t>(k_ops);
+  return s;
+}
+
+// Built-in latency model. Coefficients per (op, protocol, nranks) were fitted
+// on B200 measurements of the message-size sweep; rank counts that were not
+// measured use the nearest measured one.
+void builtin_model(sfc_cost_model* m) {
+  std::memset(m, 0, sizeof(*m));
+  for (int op = 0; op < 2; ++op)
+    for (int pr = 0; pr < SFC_NUM_PROTOCOLS; ++pr)
+      for (int n = 0; n <= SFC_MAX_RANKS; ++n) m->c[op][pr][n] = {-1.0, 0.0};
+  // alpha (us), beta (us per algorithmic byte); placeholders until fitted
+  const double a[6] = {0, 1.5, 2.5, 2.0, 3.0, 4.5};
+  const double b[6] = {0, 1.0 / 5.0e6, 1.0 / 5.0e6, 1.0 / 5.0e6, 1.0 / 5.0e6, 1.0 / 5.0e6};
+  for (int op = 0; op < 2; ++op)
+    for (int pr = 1; pr < SFC_NUM_PROTOCOLS; ++pr)
+      for (int n = kMinRanks; n <= SFC_MAX_RANKS; ++n) {
+        if (op == SFC_OP_ALLGATHER && pr == kTwoshot) continue;
+        m->c[op][pr][n] = {a[pr], b[pr]};
+      }
+}
+
+}  // namespace
+
+// ============================================================== public API
+extern "C" {
+
+const char* sfc_status_string(sfc_status s) {
+  switch (s) {
+    case SFC_OK: return "ok";
+    case SFC_ERR_INVALID: return "invalid argument";
+    case SFC_ERR_CUDA: return "CUDA runtime error";
+    case SFC_ERR_TIMEOUT: return "device wait timed out";
+    case SFC_ERR_EPOCH: return "epoch is not the next one";
+    case SFC_ERR_RESOURCES: return "ranks' CTAs cannot all be co-resident";
+    case SFC_ERR_SENTINEL_IN_INPUT: return "input contains the sentinel pattern";
+    case SFC_ERR_UNSUPPORTED: return "unsupported protocol, operation or dtype";
+    case SFC_ERR_ABORTED: return "context aborted by an earlier device error";
+  }
+  return "unknown status";
+}
+
+double sfc_algorithmic_bytes(sfc_op op, sfc_protocol protocol, size_t count, int nranks) {
+  if (nranks < kMinRanks || nranks > kMaxRanks) return -1.0;
+  const double n = nranks;
+  const double s = 2.0 * static_cast<double>(count);
+  double enc;
+  switch (protocol) {
+    case SFC_PROTO_LL: enc = 8.0 * static_cast<double>((count + 1) / 2); break;
+    case SFC_PROTO_LL128: enc = 128.0 * static_cast<double>((count + kLL128Elems - 1) / kLL128Elems); break;
+    case SFC_PROTO_SENTINEL: enc = s; break;
+    default: enc = 0.0;
+  }
+  if (protocol == SFC_PROTO_LL || protocol == SFC_PROTO_LL128 || protocol == SFC_PROTO_SENTINEL) {
+    const double reset = protocol == SFC_PROTO_SENTINEL ? (n - 1) * s : 0.0;
+    const double written = op == SFC_OP_ALLREDUCE ? s : n * s;
+    return n * (s + 2.0 * (n - 1) * enc + written + reset);
+  }
+  if (protocol == SFC_PROTO_BARRIER_ONESHOT) {
+    return op == SFC_OP_ALLREDUCE ? n * (n * s + s) : n * (n * s + n * s);
+  }
+  if (protocol == SFC_PROTO_BARRIER_TWOSHOT && op == SFC_OP_ALLREDUCE) {
+    return n * (s + s / n + s + s);
+  }
+  return -1.0;
+}
+
+void sfc_default_cost_model(sfc_cost_model* model) {
+  if (model) builtin_model(model);
+}
+
+sfc_protocol sfc_select_protocol_model(const sfc_cost_model* m, sfc_op op, size_t bytes_per_rank, int nranks) {
+  static const int order[5] = {SFC_PROTO_SENTINEL, SFC_PROTO_LL128, SFC_PROTO_LL, SFC_PROTO_BARRIER_ONESHOT,
+                               SFC_PROTO_BARRIER_TWOSHOT};
+  if (m == nullptr || nranks < kMinRanks || nranks > kMaxRanks || (op != 0 && op != 1)) return SFC_PROTO_AUTO;
+  const size_t count = bytes_per_rank / 2;
+  int best = SFC_PROTO_AUTO;
+  double best_t = 0, best_b = 0;
+  for (int i = 0; i < 5; ++i) {
+    const int pr = order[i];
+    const sfc_cost_coeff cc = m->c[op][pr][nranks];
+    if (cc.alpha_us < 0) continue;
+    const double b = sfc_algorithmic_bytes(op, static_cast<sfc_protocol>(pr), count, nranks);
+    if (b < 0) continue;
+    const double t = cc.alpha_us + cc.beta_us_per_byte * b;
+    if (best == SFC_PROTO_AUTO || t < best_t || (t == best_t && b < best_b)) {
+      best = pr;
+      best_t = t;
+      best_b = b;
+    }
+  }
+  return static_cast<sfc_protocol>(best);
+}
+
+sfc_protocol sfc_select_protocol(const sfc_ctx* c, sfc_op op, size_t bytes_per_rank, int nranks) {
+  if (c == nullptr) return SFC_PROTO_AUTO;
+  sfc_cost_model m = c->model;
+  // protocols without scratch in this context are never chosen
+  for (int pr = 1; pr < SFC_NUM_PROTOCOLS; ++pr)
+    if (!provisioned(c, pr))
+      for (int o = 0; o < 2; ++o)
+        for (int n = 0; n <= SFC_MAX_RANKS; ++n) m.c[o][pr][n].alpha_us = -1.0;
+  return sfc_select_protocol_model(&m, op, bytes_per_rank, nranks);
+}
+
+sfc_status sfc_set_cost_model(sfc_ctx* c, const sfc_cost_model* m) {
+  if (c == nullptr || m == nullptr) return SFC_ERR_INVALID;
+  c->model = *m;
+  return SFC_OK;
+}
+
+sfc_status sfc_init(sfc_ctx** out, int nranks, size_t max_bytes_per_rank, const sfc_config* cfg) {
+  if (out == nullptr) return SFC_ERR_INVALID;
+  *out = nullptr;
+  if (nranks < kMinRanks || nranks > kMaxRanks || max_bytes_per_rank == 0) return SFC_ERR_INVALID;
+  if (cfg && (cfg->ctas_per_rank < 0 || cfg->ctas_per_rank > kBarStride)) return SFC_ERR_INVALID;
+  if (cfg && (cfg->protocol_mask & ~0x3Eu)) return SFC_ERR_INVALID;
+  sfc_ctx* c = new sfc_ctx();
+  if (cfg) c->cfg = *cfg;
+  c->nranks = nranks;
+  c->max_bytes = max_bytes_per_rank;
+  c->max_count = max_bytes_per_rank / 2;
+  builtin_model(&c->model);
+  auto fail = [&](sfc_status s) {
+    sfc_destroy(c);
+    return s;
+  };
+  if (!cuda_ok(cudaGetDevice(&c->device))) return fail(SFC_ERR_CUDA);
+  if (!cuda_ok(cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, c->device)))
+    return fail(SFC_ERR_CUDA);
+  int coop = 0;
+  if (!cuda_ok(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, c->device)) || !coop)
+    return fail(SFC_ERR_UNSUPPORTED);
+  const uint64_t slots = static_cast<uint64_t>(nranks) * 2 * (nranks - 1);
+  for (int pr : {kLL, kLL128, kSentinel}) {
+    if (!provisioned(c, pr)) continue;
+    const uint64_t sb = (slot_bytes_gpu(pr, c->max_count) + 255) / 256 * 256;
+    c->slot_stride[pr] = sb;
+    c->region_bytes[pr] = sb * slots;
+    if (!cuda_ok(cudaMalloc(&c->region[pr], c->region_bytes[pr]))) return fail(SFC_ERR_CUDA);
+  }
+  c->bar_stride = kBarStride;
+  if (!cuda_ok(cudaMalloc(&c->bar, sizeof(uint64_t) * nranks * kBarStride))) return fail(SFC_ERR_CUDA);
+  if (provisioned(c, kTwoshot)) {
+    const uint64_t nvec = (c->max_count + 7) / 8;
+    c->red_stride = ((nvec + nranks - 1) / nranks) * 8;
+    if (!cuda_ok(cudaMalloc(&c->red, std::max<uint64_t>(16, 2 * c->red_stride * nranks) /* bytes */))) return fail(SFC_ERR_CUDA);
+  }
+  if (!cuda_ok(cudaMalloc(&c->dstatus, sizeof(DevStatus)))) return fail(SFC_ERR_CUDA);
+  if (!cuda_ok(cudaMallocHost(&c->hstatus, sizeof(DevStatus)))) return fail(SFC_ERR_CUDA);
+  sfc_status s = sfc_reset(c, nullptr);
+  if (s != SFC_OK) return fail(s);
+  if (!cuda_ok(cudaStreamSynchronize(nullptr))) return fail(SFC_ERR_CUDA);
+  *out = c;
+  return SFC_OK;
+}
+
+sfc_status sfc_destroy(sfc_ctx* c) {
+  if (c == nullptr) return SFC_ERR_INVALID;
+  (void)cudaDeviceSynchronize();
+  for (auto& r : c->region) {
+    if (r) cudaFree(r);
+    r = nullptr;
+  }
+  if (c->bar) cudaFree(c->bar);
+  if (c->red) cudaFree(c->red);
+  if (c->dstatus) cudaFree(c->dstatus);
+  if (c->hstatus) cudaFreeHost(c->hstatus);
+  if (c->stage_in) cudaFree(c->stage_in);
+  if (c->stage_out) cudaFree(c->stage_out);
+  delete c;
+  return SFC_OK;
+}
+
+sfc_status sfc_reset(sfc_ctx* c, void* stream) {
+  if (c == nullptr) return SFC_ERR_INVALID;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int pr : {kLL, kLL128, kSentinel}) {
+    if (c->region[pr] == nullptr) continue;
+    const int fill = pr == kSentinel ? 0xFF : 0x00;
+    if (!cuda_ok(cudaMemsetAsync(c->region[pr], fill, c->region_bytes[pr], st))) return SFC_ERR_CUDA;
+  }
+  if (!cuda_ok(cudaMemsetAsync(c->bar, 0, sizeof(uint64_t) * c->nranks * c->bar_stride, st))) return SFC_ERR_CUDA;
+  if (!cuda_ok(cudaMemsetAsync(c->dstatus, 0, sizeof(DevStatus), st))) return SFC_ERR_CUDA;
+  c->next_epoch = 1;
+  c->poisoned = false;
+  c->last_stream = st;
+  return SFC_OK;
+}
+
+sfc_status sfc_allreduce(sfc_ctx* c, const void* const* in, void* const* out, size_t count, sfc_dtype dtype,
+                         sfc_protocol protocol, uint32_t epoch, void* stream) {
+  return one_op(c, SFC_OP_ALLREDUCE, in, out, count, dtype, protocol, epoch, stream);
+}
+
+sfc_status sfc_allgather(sfc_ctx* c, const void* const* in, void* const* out, size_t count, sfc_dtype dtype,
+                         sfc_protocol protocol, uint32_t epoch, void* stream) {
+  return one_op(c, SFC_OP_ALLGATHER, in, out, count, dtype, protocol, epoch, stream);
+}
+
+sfc_status sfc_allreduce_chain(sfc_ctx* c, int k_ops, const void* const* in_table, void* const* out_table,
+                               size_t count, sfc_dtype dtype, sfc_protocol protocol, uint32_t first_epoch,
+                               const uint32_t* skew_ns, uint64_t* timings, void* stream) {
+  return chain(c, SFC_OP_ALLREDUCE, k_ops, in_table, out_table, count, dtype, protocol, first_epoch, skew_ns,
+               timings, stream);
+}
+
+sfc_status sfc_allgather_chain(sfc_ctx* c, int k_ops, const void* const* in_table, void* const* out_table,
+                               size_t count, sfc_dtype dtype, sfc_protocol protocol, uint32_t first_epoch,
+                               const uint32_t* skew_ns, uint64_t* timings, void* stream) {
+  return chain(c, SFC_OP_ALLGATHER, k_ops, in_table, out_table, count, dtype, protocol, first_epoch, skew_ns,
+               timings, stream);
+}
+
+sfc_status sfc_allreduce_chain_host(sfc_ctx* c, int k_ops, const void* in_host, void* out_host, size_t count,
+                                    sfc_dtype dtype, sfc_protocol protocol, uint32_t first_epoch, uint64_t* timings,
+                                    void* stream) {
+  if (c == nullptr || in_host == nullptr || out_host == nullptr || k_ops < 1) return SFC_ERR_INVALID;
+  if (count == 0) return dtype == SFC_BF16 ? SFC_OK : SFC_ERR_UNSUPPORTED;
+  int proto = protocol;
+  if (proto == SFC_PROTO_AUTO) proto = sfc_select_protocol(c, SFC_OP_ALLREDUCE, count * 2, c->nranks);
+  sfc_status s = check_common(c, SFC_OP_ALLREDUCE, count, dtype, proto, first_epoch, k_ops);
+  if (s != SFC_OK) return s;
+  const uint64_t stride = (count + 7) / 8 * 8;  // keep every operand 16-byte aligned
+  const size_t need = static_cast<size_t>(k_ops) * c->nranks * stride * 2;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (need > c->stage_bytes) {
+    if (c->stage_in || c->stage_out) {
+      if (!cuda_ok(cudaStreamSynchronize(st))) return SFC_ERR_CUDA;
+      cudaFree(c->stage_in);
+      cudaFree(c->stage_out);
+      c->stage_in = c->stage_out = nullptr;
+      c->stage_bytes = 0;
+    }
+    if (!cuda_ok(cudaMalloc(&c->stage_in, need)) || !cuda_ok(cudaMalloc(&c->stage_out, need))) return SFC_ERR_CUDA;
+    c->stage_bytes = need;
+  }
+  const size_t rows = static_cast<size_t>(k_ops) * c->nranks;
+  if (!cuda_ok(cudaMemcpy2DAsync(c->stage_in, stride * 2, in_host, count * 2, count * 2, rows,
+                                 cudaMemcpyHostToDevice, st)))
+    return SFC_ERR_CUDA;
+  s = prepare_timings(timings, k_ops, st);
+  if (s != SFC_OK) return s;
+  KParams p{};
+  p.addr_mode = 2;
+  p.in_base = c->stage_in;
+  p.out_base = c->stage_out;
+  p.in_stride = stride;
+  p.out_stride = stride;
+  p.timings = timings;
+  const int G = choose_G(c, proto, SFC_OP_ALLREDUCE, count, nullptr);
+  fill_common(c, p, proto, count, k_ops, first_epoch, G);
+  s = launch(c, proto, SFC_OP_ALLREDUCE, p, st);
+  if (s != SFC_OK) return s;
+  c->next_epoch = first_epoch + static_cast<uint32_t>(k_ops);
+  if (!cuda_ok(cudaMemcpy2DAsync(out_host, count * 2, c->stage_out, stride * 2, count * 2, rows,
+                                 cudaMemcpyDeviceToHost, st)))
+    return SFC_ERR_CUDA;
+  return SFC_OK;
+}
+
+sfc_status sfc_get_status(sfc_ctx* c, uint32_t* info) {
+  if (c == nullptr) return SFC_ERR_INVALID;
+  if (!cuda_ok(cudaMemcpyAsync(c->hstatus, c->dstatus, sizeof(DevStatus), cudaMemcpyDeviceToHost, c->last_stream)))
+    return SFC_ERR_CUDA;
+  if (!cuda_ok(cudaStreamSynchronize(c->last_stream))) return SFC_ERR_CUDA;
+  if (info) *info = c->hstatus->info;
+  const int code = c->hstatus->code;
+  if (code != 0 || c->hstatus->abort) c->poisoned = true;
+  if (code == 0 && c->hstatus->abort) return SFC_ERR_ABORTED;
+  return static_cast<sfc_status>(code);
+}
+
+uint32_t sfc_next_epoch(const sfc_ctx* c) { return c ? c->next_epoch : 0; }
+
+sfc_status sfc_launch_shape(sfc_ctx* c, sfc_op op, sfc_protocol protocol, size_t count, int* ctas_per_rank,
+                            int* threads_per_cta) {
+  if (c == nullptr || (op != 0 && op != 1)) return SFC_ERR_INVALID;
+  int proto = protocol;
+  if (proto == SFC_PROTO_AUTO) proto = sfc_select_protocol(c, op, count * 2, c->nranks);
+  if (proto < kLL || proto > kTwoshot) return SFC_ERR_INVALID;
+  if (kernel_for(c->nranks, proto, op) == nullptr) return SFC_ERR_UNSUPPORTED;
+  const int G = choose_G(c, proto, op, count, nullptr);
+  if (G <= 0) return SFC_ERR_RESOURCES;
+  if (ctas_per_rank) *ctas_per_rank = G;
+  if (threads_per_cta) *threads_per_cta = kThreads;
+  return SFC_OK;
+}
+
+sfc_status sfc_scratch_slot(sfc_ctx* c, sfc_protocol protocol, int rank, int parity, int src, void** ptr,
+                            size_t* bytes) {
+  if (c == nullptr || ptr == nullptr) return SFC_ERR_INVALID;
+  const int pr = protocol;
+  if (!self_sync(pr) || c->region[pr] == nullptr) return SFC_ERR_UNSUPPORTED;
+  if (rank < 0 || rank >= c->nranks || src < 0 || src >= c->nranks || src == rank || (parity != 0 && parity != 1))
+    return SFC_ERR_INVALID;
+  const int j = src < rank ? src : src - 1;
+  const uint64_t idx = static_cast<uint64_t>((rank * 2 + parity) * (c->nranks - 1) + j);
+  *ptr = c->region[pr] + idx * c->slot_stride[pr];
+  if (bytes) *bytes = c->slot_stride[pr];
+  return SFC_OK;
+}
+
+sfc_status sfc_set_silent_rank(sfc_ctx* c, int silent_rank) {
+  if (c == nullptr || silent_rank < -1 || silent_rank >= c->nranks) return SFC_ERR_INVALID;
+  c->silent_rank = silent_rank;
+  return SFC_OK;
+}
+
+uint64_t sfc_launch_count(const sfc_ctx* c) { return c ? c->launches : 0; }
+
+}  // extern "C"

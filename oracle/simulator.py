@@ -66,7 +66,7 @@ from . import protocols as P
 from . import reference
 from .bf16 import BF16_SENTINEL, bf16_bits_to_f32, f32_to_bf16_bits
 
-__all__ = ["ChainSim", "run_chain", "BARRIER_ONESHOT", "BARRIER_TWOSHOT", "ALL_PROTOCOLS"]
+__all__ = ["ChainSim", "run_chain", "run_fifo", "BARRIER_ONESHOT", "BARRIER_TWOSHOT", "ALL_PROTOCOLS"]
 
 BARRIER_ONESHOT = "barrier_oneshot"
 BARRIER_TWOSHOT = "barrier_twoshot"
@@ -472,6 +472,31 @@ class ChainSim:
                         v.append(f"slot {(r, par, q)} unit {j} flag is not epoch {last[par]}")
                         break
         return v
+
+
+def run_fifo(proto, inputs, op=ALLREDUCE, first_epoch=1):
+    """One fixed, cheap schedule for large inputs: in rounds, every rank
+    that can push pushes, every pending store lands in issue order, every
+    rank polls. Linear in the number of units; returns (sim, violations)."""
+    sim = ChainSim(proto, inputs, op=op, first_epoch=first_epoch)
+    while not sim.finished():
+        progressed = False
+        for r in range(sim.N):
+            if sim.ranks[r].phase != "done" and (proto not in P.SELF_SYNC or sim.ranks[r].phase == "push"):
+                if proto in P.SELF_SYNC or sim._barrier_can_step(r):
+                    sim.apply(("step", r))
+                    progressed = True
+        while sim.pending:
+            sim.apply(("land", 0))
+            progressed = True
+        if proto in P.SELF_SYNC:
+            for r in range(sim.N):
+                if sim.ranks[r].phase == "poll" and sim._poll_would_progress(r):
+                    sim.apply(("step", r))
+                    progressed = True
+        if not progressed:
+            break
+    return sim, sim.final_checks()
 
 
 def run_chain(proto, inputs, op=ALLREDUCE, first_epoch=1, schedule="random", seed=0,

@@ -128,3 +128,10 @@ def test_first_epoch_and_parity_offset():
     x = _x(22, 4, 3, 5)
     _, v = S.run_chain(P.LL, x, first_epoch=1000, seed=1)
     assert not v
+
+
+@pytest.mark.parametrize("proto", SELF + [S.BARRIER_ONESHOT, S.BARRIER_TWOSHOT])
+def test_fifo_schedule_for_large_inputs(proto):
+    x = _x(23, 2, 4, 300)
+    _, v = S.run_fifo(proto, x)
+    assert not v, v[:3]
