@@ -46,6 +46,19 @@ def _dist():
     return ws, rank, local
 
 
+def reduce_max_over_ranks(values, device=None):
+    """Element-wise maximum of a list of floats over all processes (the
+    replicas' reported latencies); the identity with one process."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 def _percentile(v, q):
     v = sorted(v)
     if not v:
@@ -288,10 +301,7 @@ def run_gpu(args):
 
     head = per_size[0]
     value = head["p50_us"]
-    if ws > 1:
-        tv = torch.tensor([value, e2e_us], dtype=torch.float64, device=dev)
-        dist.all_reduce(tv, op=dist.ReduceOp.MAX)
-        value, e2e_us = float(tv[0]), float(tv[1])
+    value, e2e_us = reduce_max_over_ranks([value, e2e_us], device=dev)
 
     dom = per_size[-1]  # largest size: most time per step
     ach = dom["achieved_gbs_launch"]
