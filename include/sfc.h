@@ -235,6 +235,30 @@ sfc_status sfc_measure_floor(int iters, sfc_floor_result* out);
 /* Number of kernel launches this context has issued (all entry points). */
 uint64_t sfc_launch_count(const sfc_ctx* ctx);
 
+/* Largest per-rank element count sfc_allreduce_noalloc accepts (8 KB of bf16). */
+#define SFC_NOALLOC_MAX_COUNT 4096
+
+/* One LL all-reduce that allocates nothing. The pages have no counterpart:
+ * this is a library convenience for callers that cannot call cudaMalloc when
+ * they need the collective -- code inside an allocator or an out-of-memory
+ * path, a process that reserved all device memory at start-up, or a host
+ * library that may not own allocations. Its scratch is a file-scope static
+ * device array of about 1.8 MB that every GPU loading this library keeps until
+ * the process exits; no context is needed.
+ *   in / out: HOST arrays of `nranks` (2..8) DEVICE pointers, 16-byte
+ *   aligned, `count` bf16 elements each, no overlap; result as sfc_allreduce
+ *   (rank-order fp32 sum, one bf16 rounding), every rank the same bits.
+ *   count > SFC_NOALLOC_MAX_COUNT -> SFC_ERR_INVALID; count == 0 -> no-op.
+ * Each call clears the part of the array it uses (cudaMemsetAsync on
+ * `stream`), then launches; it calls no cudaMalloc, cudaFree or allocating
+ * library routine. The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current: make that first
+ * call before any stream capture. All calls share the one array and it keeps
+ * the last call's contents, so calls that overlap on the GPU (other streams,
+ * other threads) race: order them. Device-side errors are not reported. */
+sfc_status sfc_allreduce_noalloc(const void* const* in, void* const* out, int nranks, size_t count,
+                                 void* stream);
+
 #ifdef __cplusplus
 }
 #endif
