@@ -192,7 +192,7 @@ def run_gpu(args):
     peaks = _peaks()
     max_count = HIDDEN * max(TOKENS)
     comm = api.Communicator(NRANKS, max_count * 2, protocols=[PROTOCOL, "ll", "ll128"])
-    floor = api.measure_floor(20000)
+    floor = api.measure_floor(4000)
 
     # operands: 160 distinct inputs per rank, outputs alternate two buffers
     chains = []
@@ -322,6 +322,9 @@ def run_gpu(args):
             "config": _config(), "per_size": per_size,
             "floor": {"flag_rtt_us_p50": floor["flag_rtt_ns_p50"] / 1e3,
                       "flag_rtt_us_p99": floor["flag_rtt_ns_p99"] / 1e3,
+                      "flag_rtt_us_fastest_pair": floor["flag_rtt_ns_min_pair"] / 1e3,
+                      "flag_rtt_us_slowest_pair": floor["flag_rtt_ns_max_pair"] / 1e3,
+                      "sm_pairs": floor["pairs"],
                       "l2_rtt_us": floor["l2_rtt_ns_p50"] / 1e3,
                       "sol_analogue_us": (2 * floor["l2_rtt_ns_p50"] + floor["flag_rtt_ns_p50"] / 2) / 1e3,
                       "globaltimer_step_ns": floor["globaltimer_step_ns"], "sm_clock_ghz": floor["sm_clock_ghz"],

@@ -105,8 +105,12 @@ typedef struct {
 } sfc_cost_model;
 
 typedef struct {
-  double flag_rtt_ns_p50;   /* two CTAs on different SMs ping-pong a flag */
+  double flag_rtt_ns_p50;   /* two CTAs on different SMs ping-pong a flag; median
+                               over all round trips of 16 SM pairs */
   double flag_rtt_ns_p99;
+  double flag_rtt_ns_min_pair; /* median of the fastest / slowest SM pair */
+  double flag_rtt_ns_max_pair;
+  int pairs;
   double l2_rtt_ns_p50;     /* dependent L2-hit loads, one thread */
   double sm_clock_ghz;      /* clock64 ticks per globaltimer ns during the run */
   double globaltimer_step_ns; /* smallest nonzero globaltimer increment seen */

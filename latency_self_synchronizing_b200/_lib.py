@@ -9,7 +9,8 @@ import ctypes as C
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libsfc.so")
+# SFC_LIB selects another build of the same library (e.g. a debug build).
+LIB_PATH = os.environ.get("SFC_LIB") or os.path.join(_HERE, "libsfc.so")
 
 SFC_NUM_PROTOCOLS = 6
 SFC_MAX_RANKS = 8
@@ -30,6 +31,7 @@ class CostModel(C.Structure):
 
 class FloorResult(C.Structure):
     _fields_ = [("flag_rtt_ns_p50", C.c_double), ("flag_rtt_ns_p99", C.c_double),
+                ("flag_rtt_ns_min_pair", C.c_double), ("flag_rtt_ns_max_pair", C.c_double), ("pairs", C.c_int),
                 ("l2_rtt_ns_p50", C.c_double), ("sm_clock_ghz", C.c_double),
                 ("globaltimer_step_ns", C.c_double), ("sm_a", C.c_int), ("sm_b", C.c_int)]
 

@@ -77,6 +77,12 @@ SFC_DEV int ld_rlx_s32(const void* p) {
   asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
+// Atomic exchange (relaxed, gpu scope): returns the old 8 bytes, leaves v.
+SFC_DEV uint64_t atom_exch_u64(void* p, uint64_t v) {
+  uint64_t old;
+  asm volatile("atom.relaxed.gpu.global.exch.b64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+  return old;
+}
 // ---- release / acquire -----------------------------------------------------
 SFC_DEV void st_rel_u64(void* p, uint64_t v) {
   asm volatile("st.release.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
@@ -104,6 +110,9 @@ SFC_DEV uint32_t ld_nc_u16(const void* p) {
   asm("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
   return v;
 }
+// Bring the line holding p into L2 (no register result).
+SFC_DEV void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 template <typename T>
 SFC_DEV T ld_nc_ptr(const T* p) {
   uint64_t v;

@@ -6,7 +6,8 @@
 //  * flag round trip: two CTAs on different SMs (each asks for more than half
 //    of an SM's shared memory, so they cannot share one) ping-pong a 64-bit
 //    flag with relaxed gpu-scope stores and polls; the initiator times each
-//    round trip with clock64.
+//    round trip with clock64. Repeated for 16 responder SMs spread over the
+//    GPU (both dies), so the median covers near and far pairs.
 //  * L2 round trip: one thread chases a pointer chain through a small buffer
 //    with L1-bypassing loads, so every load is one L2 hit.
 // Every wait is bounded by a %globaltimer deadline.
@@ -24,13 +25,17 @@ namespace {
 constexpr uint64_t kFloorTimeoutNs = 200ull * 1000 * 1000;  // 200 ms per trial
 constexpr int kFloorSmem = 160 * 1024;
 
-__global__ void flag_pingpong(uint64_t* flags, int iters, uint64_t* cycles, uint64_t* cal, int* sms, int* err) {
+// Grid of one CTA per SM (each asks for more than half of an SM's shared
+// memory). CTA 0 is the initiator, CTA `responder` answers, all others exit.
+__global__ void flag_pingpong(uint64_t* flags, int iters, int responder, uint64_t* cycles, uint64_t* cal,
+                              int* sms, int* err) {
   extern __shared__ uint8_t keep_apart[];
   if (threadIdx.x != 0) return;
+  if (blockIdx.x != 0 && blockIdx.x != static_cast<unsigned>(responder)) return;
   keep_apart[0] = 0;
   uint64_t* a = flags;       // initiator -> responder
   uint64_t* b = flags + 32;  // responder -> initiator (another 256-byte block)
-  sms[blockIdx.x] = static_cast<int>(smid());
+  sms[blockIdx.x == 0 ? 0 : 1] = static_cast<int>(smid());
   const uint64_t deadline = gtimer() + kFloorTimeoutNs;
   if (blockIdx.x == 0) {
     const uint64_t g0 = gtimer();
@@ -114,8 +119,19 @@ double pct(std::vector<uint64_t> v, double q) {
 extern "C" sfc_status sfc_measure_floor(int iters, sfc_floor_result* out) {
   using namespace sfc;
   if (out == nullptr || iters < 16 || iters > (1 << 20)) return SFC_ERR_INVALID;
-  const int trials = 4;
-  const int chain_n = 4096;  // 32 KB chain: L2 resident, far larger than nothing else
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SFC_ERR_CUDA;
+  }
+  int sm_count = 0;
+  if (cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sm_count < 2) {
+    (void)cudaGetLastError();
+    return SFC_ERR_CUDA;
+  }
+  // responders spread over the grid: pairs on the same and on different dies
+  const int trials = std::min(16, sm_count - 1);
+  const int chain_n = 4096;  // 32 KB pointer chain: L2 resident
   uint64_t* dflags = nullptr;
   uint64_t* dcycles = nullptr;
   uint64_t* dcal = nullptr;
@@ -125,6 +141,7 @@ extern "C" sfc_status sfc_measure_floor(int iters, sfc_floor_result* out) {
   uint64_t* dout = nullptr;
   sfc_status st = SFC_OK;
   std::vector<uint64_t> rtts;
+  std::vector<double> pair_p50;
   std::vector<uint64_t> hcal(2 * trials);
   int hsms[2] = {0, 0};
   int herr = 0;
@@ -152,13 +169,15 @@ extern "C" sfc_status sfc_measure_floor(int iters, sfc_floor_result* out) {
     }
     std::vector<uint64_t> hcycles(iters);
     for (int t = 0; t < trials && st == SFC_OK; ++t) {
+      int responder = 1 + static_cast<int>((static_cast<int64_t>(t) * (sm_count - 1)) / trials);
+      if (responder >= sm_count) responder = sm_count - 1;
       if (!ok(cudaMemset(dflags, 0, 64 * sizeof(uint64_t))) || !ok(cudaMemset(derr, 0, sizeof(int)))) {
         st = SFC_ERR_CUDA;
         break;
       }
-      void* args[] = {&dflags, &iters, &dcycles, &dcal, &dsms, &derr};
-      if (!ok(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(&flag_pingpong), dim3(2), dim3(32), args,
-                                          kFloorSmem, nullptr)) ||
+      void* args[] = {&dflags, &iters, &responder, &dcycles, &dcal, &dsms, &derr};
+      if (!ok(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(&flag_pingpong), dim3(sm_count), dim3(32),
+                                          args, kFloorSmem, nullptr)) ||
           !ok(cudaDeviceSynchronize())) {
         st = SFC_ERR_CUDA;
         break;
@@ -175,7 +194,9 @@ extern "C" sfc_status sfc_measure_floor(int iters, sfc_floor_result* out) {
         break;
       }
       // the first iterations warm the lines; keep the rest
-      rtts.insert(rtts.end(), hcycles.begin() + std::min(iters / 8, 64), hcycles.end());
+      std::vector<uint64_t> kept(hcycles.begin() + std::min(iters / 8, 64), hcycles.end());
+      pair_p50.push_back(pct(kept, 0.5));
+      rtts.insert(rtts.end(), kept.begin(), kept.end());
     }
     if (st != SFC_OK) break;
     std::vector<uint64_t> hchain(chain_n);
@@ -201,6 +222,9 @@ extern "C" sfc_status sfc_measure_floor(int iters, sfc_floor_result* out) {
     out->sm_clock_ghz = ghz;
     out->flag_rtt_ns_p50 = pct(rtts, 0.50) / ghz;
     out->flag_rtt_ns_p99 = pct(rtts, 0.99) / ghz;
+    out->flag_rtt_ns_min_pair = *std::min_element(pair_p50.begin(), pair_p50.end()) / ghz;
+    out->flag_rtt_ns_max_pair = *std::max_element(pair_p50.begin(), pair_p50.end()) / ghz;
+    out->pairs = static_cast<int>(pair_p50.size());
     out->l2_rtt_ns_p50 = static_cast<double>(chase[0]) / steps / ghz;
     out->globaltimer_step_ns = static_cast<double>(step);
     out->sm_a = hsms[0];

@@ -7,12 +7,26 @@
 // operation e, then polls the same elements from every peer, and the peers'
 // threads with the same index do the same. A writer reaches epoch e+2 only
 // after the reader's epoch e+1 push arrived, which the reader issues only
-// after it consumed epoch e (and, for the sentinel, rewrote the slot); a
-// fence.acq_rel.gpu between the end of one operation and the pushes of the
-// next makes that ordering hold in the memory model. That is the double
-// buffering of "Why Microseconds Matter in AI Infrastructure", section
-// "Latency can matter more than bandwidth": receipt of data is the evidence
-// that the other buffer can be reused, with no global barrier.
+// after it consumed epoch e. That is the double buffering of "Why
+// Microseconds Matter in AI Infrastructure", section "Latency can matter more
+// than bandwidth": receipt of data is the evidence that the other buffer can
+// be reused, with no global barrier.
+//
+// Why no fence is needed between one operation's reads and the next one's
+// pushes (a fence.acq_rel.gpu costs about 0.6 us on B200 even with nothing
+// outstanding):
+//  * LL and sentinel: the reader's next push is control dependent on the
+//    poll accesses that returned epoch e's data (the poll loop exits on their
+//    values), and the writer's e+2 store is control dependent on observing
+//    that push. For the writer's e+2 store to be seen by (or, for the
+//    sentinel's exchange, to precede) the reader's epoch-e access, the cycle
+//    access(e) -> push(e+1) -> poll(e+1) -> store(e+2) -> access(e) through
+//    dependencies and reads-from would have to exist, which the PTX memory
+//    model's no-thin-air axiom excludes.
+//  * Sentinel: the reset is the write half of the atomic exchange that reads
+//    the data, so it is ordered with the data by atomicity, not by a fence.
+//  * LL128: the writer's release fence between data and flags also orders
+//    every earlier read of the thread before its next flags.
 //
 // Within an operation a warp polls all its sources at once (independent
 // loads, one round trip per poll) and the warp decides with a vote whether
@@ -46,6 +60,25 @@ SFC_DEV uint8_t* slot_ptr(const KParams& p, int recv, int par, int src) {
   return p.scratch + static_cast<uint64_t>((recv * 2 + par) * (N - 1) + j) * p.slot_stride;
 }
 
+// The next operation's input is brought into L2 while this one is in flight,
+// standing in for a decode layer whose freshly produced activation sits in L2
+// when its all-reduce starts; its values are read only after this operation
+// completes. Each rank touches its own input: up to 8 of the thread's
+// vectors (every small message; the head of a large one).
+SFC_DEV void prefetch_next_input(const uint16_t* nx, uint64_t gtid, uint64_t gstride, uint64_t nvec) {
+  if (nx == nullptr) return;
+  int n = 0;
+  for (uint64_t v = gtid; v < nvec && n < 8; v += gstride, ++n) prefetch_l2(nx + v * 8);
+}
+
+// Operand pointers of the current operation and the next input, read one
+// operation ahead so that no table load sits on an operation's critical path.
+struct Operands {
+  const uint16_t* in;
+  uint16_t* out;
+  const uint16_t* in_next;  // null on the last operation
+};
+
 SFC_DEV uint64_t ll_off(uint64_t v, int half) {
   return ((v >> 5) << 10) + (static_cast<uint64_t>(half) << 9) + ((v & 31) << 4);
 }
@@ -78,14 +111,14 @@ struct PendingOut {
 // the two loads equal e.
 template <int N, int OP>
 SFC_DEV bool ll_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid, uint64_t gstride,
-                   PendingOut& pend) {
+                   const Operands& io, PendingOut& pend) {
   const uint64_t count = p.count;
   const uint64_t nvec = (count + 7) >> 3;
   const int par = e & 1;
   const uint64_t ehi = static_cast<uint64_t>(e) << 32;
   const int lane = threadIdx.x & 31;
-  const uint16_t* in_r = in_ptr<N>(p, op, r);
-  uint16_t* out_r = out_ptr<N>(p, op, r);
+  const uint16_t* in_r = io.in;
+  uint16_t* out_r = io.out;
 
   if (r != p.silent_rank) {
     for (uint64_t v = gtid; v < nvec; v += gstride) {
@@ -101,40 +134,50 @@ SFC_DEV bool ll_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid, u
     }
   }
   pend.flush();
+  prefetch_next_input(io.in_next, gtid, gstride, nvec);
 
   const uint8_t* my = slot_ptr<N>(p, r, par, r == 0 ? 1 : 0);  // slot j = 0
   for (uint64_t vb = gtid - lane; vb < nvec; vb += gstride) {
     const uint64_t v = vb + lane;
     const bool act = v < nvec;
-    uint4 x[N];
     const uint4 own = act ? load8(in_r, v * 8, count) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int q = 0; q < N; ++q) x[q] = own;
     uint32_t need = act ? (((1u << N) - 1u) & ~(1u << r)) : 0u;
     const uint64_t o0 = ll_off(v, 0), o1 = ll_off(v, 1);
+    // a source's registers keep the units that validated: once accepted it is
+    // not loaded again
+    uint64_t a[N], b[N], c[N], d[N];
     WarpWait ww;
     while (true) {
+      // issue every pending source's loads before looking at any result, so
+      // one poll costs one round trip whatever the number of sources
+      const uint32_t cur = need;
 #pragma unroll
       for (int q = 0; q < N; ++q) {
-        if (need & (1u << q)) {
+        if (cur & (1u << q)) {
           const int j = q < r ? q : q - 1;
           const uint8_t* s = my + static_cast<uint64_t>(j) * p.slot_stride;
-          uint64_t a, b, c, d;
-          ld_rlx_v2u64(s + o0, a, b);
-          ld_rlx_v2u64(s + o1, c, d);
-          const bool ok = static_cast<uint32_t>(a >> 32) == e && static_cast<uint32_t>(b >> 32) == e &&
-                          static_cast<uint32_t>(c >> 32) == e && static_cast<uint32_t>(d >> 32) == e;
-          if (ok) {
-            x[q] = make_uint4(static_cast<uint32_t>(a), static_cast<uint32_t>(b), static_cast<uint32_t>(c),
-                              static_cast<uint32_t>(d));
-            need &= ~(1u << q);
-          }
+          ld_rlx_v2u64(s + o0, a[q], b[q]);
+          ld_rlx_v2u64(s + o1, c[q], d[q]);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < N; ++q) {
+        if (cur & (1u << q)) {
+          const bool ok = static_cast<uint32_t>(a[q] >> 32) == e && static_cast<uint32_t>(b[q] >> 32) == e &&
+                          static_cast<uint32_t>(c[q] >> 32) == e && static_cast<uint32_t>(d[q] >> 32) == e;
+          if (ok) need &= ~(1u << q);
         }
       }
       if (!__any_sync(kFull, need != 0u)) break;
       if (ww.tick(p, op, r, need ? __ffs(need) - 1 : -1)) return false;
     }
     if (act) {
+      uint4 x[N];
+#pragma unroll
+      for (int q = 0; q < N; ++q)
+        x[q] = q == r ? own
+                      : make_uint4(static_cast<uint32_t>(a[q]), static_cast<uint32_t>(b[q]),
+                                   static_cast<uint32_t>(c[q]), static_cast<uint32_t>(d[q]));
       if (OP == kAllreduce) {
         pend.set(out_r, v * 8, reduce8<N>(x), count);
       } else {
@@ -147,63 +190,80 @@ SFC_DEV bool ll_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid, u
 }
 
 // ================================================================ sentinel
-// Raw 16-byte vectors into a slot pre-filled with 0xFFFF; a vector is ready
-// when none of its 8 elements is 0xFFFF; after consuming, the reader writes
-// 0xFFFF back before its next push (ordered by the per-operation fence).
+// Raw data into a slot pre-filled with 0xFFFF. The writer moves each 8 bytes
+// as one single-copy-atomic .b64 element, so an 8-byte unit of the slot is
+// either all fill or all data, and data never equals the fill (inputs never
+// hold 0xFFFF elements). The reader polls each 8-byte unit with an atomic
+// exchange against the fill: a result other than the fill is the data, and
+// the same atomic operation has already written the fill back (the reset).
 template <int N, int OP>
 SFC_DEV bool sentinel_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid, uint64_t gstride,
-                         PendingOut& pend) {
+                         const Operands& io, PendingOut& pend) {
+  constexpr uint64_t kFill = ~0ull;
   const uint64_t count = p.count;
   const uint64_t nvec = (count + 7) >> 3;
   const int par = e & 1;
   const int lane = threadIdx.x & 31;
-  const uint16_t* in_r = in_ptr<N>(p, op, r);
-  uint16_t* out_r = out_ptr<N>(p, op, r);
+  const uint16_t* in_r = io.in;
+  uint16_t* out_r = io.out;
 
   if (r != p.silent_rank) {
     for (uint64_t v = gtid; v < nvec; v += gstride) {
       const uint4 x = load8(in_r, v * 8, count);
-      // the receivers of a sentinel element would never see it arrive: record
+      // the receivers of a sentinel element may never see it arrive: record
       // the error; every wait then sees the abort word and exits
       if (p.debug && has_sentinel(x)) record_error(p, 6 /* SFC_ERR_SENTINEL_IN_INPUT */, err_info(op, r, r));
+      const uint64_t lo = (static_cast<uint64_t>(x.y) << 32) | x.x;
+      const uint64_t hi = (static_cast<uint64_t>(x.w) << 32) | x.z;
 #pragma unroll
       for (int q = 0; q < N; ++q) {
         if (q == r) continue;
-        st_rlx_v4u32(slot_ptr<N>(p, q, par, r) + v * 16, x);
+        st_rlx_v2u64(slot_ptr<N>(p, q, par, r) + v * 16, lo, hi);
       }
     }
   }
   pend.flush();
+  prefetch_next_input(io.in_next, gtid, gstride, nvec);
 
-  const uint8_t* my = slot_ptr<N>(p, r, par, r == 0 ? 1 : 0);
-  const uint4 fill = make_uint4(kFull, kFull, kFull, kFull);
+  uint8_t* my = slot_ptr<N>(p, r, par, r == 0 ? 1 : 0);
   for (uint64_t vb = gtid - lane; vb < nvec; vb += gstride) {
     const uint64_t v = vb + lane;
     const bool act = v < nvec;
-    uint4 x[N];
     const uint4 own = act ? load8(in_r, v * 8, count) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int q = 0; q < N; ++q) x[q] = own;
-    uint32_t need = act ? (((1u << N) - 1u) & ~(1u << r)) : 0u;
-    WarpWait ww;
-    while (true) {
-#pragma unroll
-      for (int q = 0; q < N; ++q) {
-        if (need & (1u << q)) {
-          const int j = q < r ? q : q - 1;
-          const uint4 y = ld_rlx_v4u32(my + static_cast<uint64_t>(j) * p.slot_stride + v * 16);
-          if (!has_sentinel(y)) {
-            x[q] = y;
-            need &= ~(1u << q);
-          }
-        }
-      }
-      if (!__any_sync(kFull, need != 0u)) break;
-      if (ww.tick(p, op, r, need ? __ffs(need) - 1 : -1)) return false;
-    }
+    // two bits per source: low and high 8-byte unit of the vector
+    uint32_t need = 0;
     if (act) {
 #pragma unroll
-      for (int j = 0; j < N - 1; ++j) st_rlx_v4u32(const_cast<uint8_t*>(my) + j * p.slot_stride + v * 16, fill);
+      for (int q = 0; q < N; ++q)
+        if (q != r) need |= 3u << (2 * q);
+    }
+    uint64_t a[N], b[N];  // keep the accepted units (never exchanged again)
+    WarpWait ww;
+    while (true) {
+      // every pending exchange is issued before any result is examined
+      const uint32_t cur = need;
+#pragma unroll
+      for (int q = 0; q < N; ++q) {
+        const int j = q < r ? q : q - 1;
+        uint8_t* s = my + static_cast<uint64_t>(j) * p.slot_stride + v * 16;
+        if (cur & (1u << (2 * q))) a[q] = atom_exch_u64(s, kFill);
+        if (cur & (2u << (2 * q))) b[q] = atom_exch_u64(s + 8, kFill);
+      }
+#pragma unroll
+      for (int q = 0; q < N; ++q) {
+        if ((cur & (1u << (2 * q))) && a[q] != kFill) need &= ~(1u << (2 * q));
+        if ((cur & (2u << (2 * q))) && b[q] != kFill) need &= ~(2u << (2 * q));
+      }
+      if (!__any_sync(kFull, need != 0u)) break;
+      if (ww.tick(p, op, r, need ? (__ffs(need) - 1) / 2 : -1)) return false;
+    }
+    if (act) {
+      uint4 x[N];
+#pragma unroll
+      for (int q = 0; q < N; ++q)
+        x[q] = q == r ? own
+                      : make_uint4(static_cast<uint32_t>(a[q]), static_cast<uint32_t>(a[q] >> 32),
+                                   static_cast<uint32_t>(b[q]), static_cast<uint32_t>(b[q] >> 32));
       if (OP == kAllreduce) {
         pend.set(out_r, v * 8, reduce8<N>(x), count);
       } else {
@@ -226,11 +286,12 @@ SFC_DEV bool sentinel_op(const KParams& p, int r, int op, uint32_t e, uint64_t g
 // once.
 template <int N>
 struct LL128Batch {
-  static constexpr int B = 32 / N;  // bits b * N + q of one 32-bit mask
+  static constexpr int B = N >= 16 ? 1 : 16 / N;  // B * N <= 16 flags in flight per lane
 };
 
 template <int N, int OP>
-SFC_DEV bool ll128_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid, uint64_t gstride) {
+SFC_DEV bool ll128_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid, uint64_t gstride,
+                      const Operands& io) {
   constexpr int B = LL128Batch<N>::B;
   const uint64_t count = p.count;
   const uint64_t nlines = (count + kLL128Elems - 1) / kLL128Elems;
@@ -240,8 +301,8 @@ SFC_DEV bool ll128_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid
   const int sub = lane & 7;
   const uint64_t lsel = static_cast<uint64_t>(lane >> 3);
   const uint64_t wg = gtid >> 5, wstride = gstride >> 5;
-  const uint16_t* in_r = in_ptr<N>(p, op, r);
-  uint16_t* out_r = out_ptr<N>(p, op, r);
+  const uint16_t* in_r = io.in;
+  uint16_t* out_r = io.out;
   const uint32_t peers = ((1u << N) - 1u) & ~(1u << r);
 
   if (r != p.silent_rank) {
@@ -275,6 +336,15 @@ SFC_DEV bool ll128_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid
       }
     }
   }
+  if (io.in_next != nullptr) {
+    const uint16_t* nx = io.in_next;
+    int n = 0;
+    for (uint64_t g = wg; g < ngroups && n < 8; g += wstride, ++n) {
+      const uint64_t L = g * kLL128LinesPerWarp + lsel;
+      const uint64_t e0 = L * kLL128Elems + sub * 8;
+      if (L < nlines && e0 < count) prefetch_l2(nx + e0);
+    }
+  }
 
   const uint8_t* my = slot_ptr<N>(p, r, par, r == 0 ? 1 : 0);
   for (uint64_t g0 = wg; g0 < ngroups; g0 += wstride * B) {
@@ -289,18 +359,23 @@ SFC_DEV bool ll128_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid
     }
     WarpWait ww;
     while (true) {
+      // all pending flags of the batch are loaded before any is compared
+      const uint32_t cur = need;
+      uint64_t f[B * N];
 #pragma unroll
       for (int b = 0; b < B; ++b) {
         const uint64_t L = (g0 + b * wstride) * kLL128LinesPerWarp + lsel;
 #pragma unroll
         for (int q = 0; q < N; ++q) {
-          if (need & (1u << (b * N + q))) {
+          if (cur & (1u << (b * N + q))) {
             const int j = q < r ? q : q - 1;
-            const uint64_t f = ld_rlx_u64(my + static_cast<uint64_t>(j) * p.slot_stride + L * kLL128Line + 120);
-            if (f == static_cast<uint64_t>(e)) need &= ~(1u << (b * N + q));
+            f[b * N + q] = ld_rlx_u64(my + static_cast<uint64_t>(j) * p.slot_stride + L * kLL128Line + 120);
           }
         }
       }
+#pragma unroll
+      for (int i = 0; i < B * N; ++i)
+        if ((cur & (1u << i)) && f[i] == static_cast<uint64_t>(e)) need &= ~(1u << i);
       if (!__any_sync(kFull, need != 0u)) break;
       if (ww.tick(p, op, r, -1)) return false;
     }
@@ -370,12 +445,14 @@ SFC_DEV bool cta_barrier(const KParams& p, int r, int k, int op, uint64_t target
 // order (all-gather: copy), bottom barrier ("SiFAR: Synchronization-Free
 // All-Reduce for Low-Latency LLM Inference", abstract).
 template <int N, int OP>
-SFC_DEV bool oneshot_op(const KParams& p, int r, int k, int op, uint32_t e, uint64_t gtid, uint64_t gstride) {
+SFC_DEV bool oneshot_op(const KParams& p, int r, int k, int op, uint32_t e, uint64_t gtid, uint64_t gstride,
+                        const Operands& io) {
   const uint64_t count = p.count;
   const uint64_t nvec = (count + 7) >> 3;
   const uint64_t eb = static_cast<uint64_t>(e) << 2;
   if (!cta_barrier<N>(p, r, k, op, eb | kPhaseTop)) return false;
-  uint16_t* out_r = out_ptr<N>(p, op, r);
+  prefetch_next_input(io.in_next, gtid, gstride, nvec);
+  uint16_t* out_r = io.out;
   const uint16_t* src[N];
 #pragma unroll
   for (int q = 0; q < N; ++q) src[q] = in_ptr<N>(p, op, q);
@@ -399,13 +476,15 @@ SFC_DEV bool oneshot_op(const KParams& p, int r, int k, int op, uint32_t e, uint
 // of each rank covers the same vector offsets inside every shard, so the
 // per-CTA-index barriers order each producer before its consumers.
 template <int N>
-SFC_DEV bool twoshot_op(const KParams& p, int r, int k, int op, uint32_t e, uint64_t gtid, uint64_t gstride) {
+SFC_DEV bool twoshot_op(const KParams& p, int r, int k, int op, uint32_t e, uint64_t gtid, uint64_t gstride,
+                        const Operands& io) {
   const uint64_t count = p.count;
   const uint64_t nvec = (count + 7) >> 3;
   const uint64_t sv = (nvec + N - 1) / N;  // vectors per shard
   const uint64_t eb = static_cast<uint64_t>(e) << 2;
   if (!cta_barrier<N>(p, r, k, op, eb | kPhaseTop)) return false;
-  uint16_t* out_r = out_ptr<N>(p, op, r);
+  prefetch_next_input(io.in_next, gtid, gstride, nvec);
+  uint16_t* out_r = io.out;
   {
     const uint16_t* src[N];
 #pragma unroll
@@ -447,25 +526,26 @@ __global__ void __launch_bounds__(kThreads, 2) sfc_kernel(const __grid_constant_
   if (p.timings != nullptr && lane == 0)
     atomicMin(reinterpret_cast<unsigned long long*>(&p.timings[0]), static_cast<unsigned long long>(gtimer()));
   PendingOut pend;
+  Operands io{in_ptr<N>(p, 0, r), out_ptr<N>(p, 0, r), nullptr};
   for (int op = 0; op < p.k_ops; ++op) {
     const uint32_t e = p.first_epoch + static_cast<uint32_t>(op);
-    if (PROTO == kLL || PROTO == kLL128 || PROTO == kSentinel) {
-      // end of the previous operation's reads / resets before these pushes
-      if (op > 0) fence_acq_rel();
-    }
+    io.in_next = op + 1 < p.k_ops ? in_ptr<N>(p, op + 1, r) : nullptr;
+    uint16_t* out_next = op + 1 < p.k_ops ? out_ptr<N>(p, op + 1, r) : nullptr;
     if (p.skew != nullptr) spin_ns(__ldg(&p.skew[op * N + r]), p.timeout_ns);
     bool ok;
     if (PROTO == kLL)
-      ok = ll_op<N, OP>(p, r, op, e, gtid, gstride, pend);
+      ok = ll_op<N, OP>(p, r, op, e, gtid, gstride, io, pend);
     else if (PROTO == kSentinel)
-      ok = sentinel_op<N, OP>(p, r, op, e, gtid, gstride, pend);
+      ok = sentinel_op<N, OP>(p, r, op, e, gtid, gstride, io, pend);
     else if (PROTO == kLL128)
-      ok = ll128_op<N, OP>(p, r, op, e, gtid, gstride);
+      ok = ll128_op<N, OP>(p, r, op, e, gtid, gstride, io);
     else if (PROTO == kOneshot)
-      ok = oneshot_op<N, OP>(p, r, k, op, e, gtid, gstride);
+      ok = oneshot_op<N, OP>(p, r, k, op, e, gtid, gstride, io);
     else
-      ok = twoshot_op<N>(p, r, k, op, e, gtid, gstride);
+      ok = twoshot_op<N>(p, r, k, op, e, gtid, gstride, io);
     if (!ok) return;
+    io.in = io.in_next;
+    io.out = out_next;
     if (p.timings != nullptr && lane == 0)
       atomicMax(reinterpret_cast<unsigned long long*>(&p.timings[1 + op]), static_cast<unsigned long long>(gtimer()));
   }

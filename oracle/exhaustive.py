@@ -136,9 +136,10 @@ def arrival_orders(inputs, bug=None):
     return combos, violations
 
 
-def explore_interleavings(proto, inputs, op="allreduce", bug=None, max_states=2_000_000):
+def explore_interleavings(proto, inputs, op="allreduce", bug=None, max_states=2_000_000,
+                          sentinel_reset="after_all"):
     """Depth-first search over all interleavings; returns (states, violations)."""
-    root = ChainSim(proto, inputs, op=op, bug=bug)
+    root = ChainSim(proto, inputs, op=op, bug=bug, sentinel_reset=sentinel_reset)
     seen = set()
     stack = [root]
     violations = []

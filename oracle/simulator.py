@@ -100,8 +100,14 @@ class ChainSim:
     ``"allreduce"`` or ``"allgather"``.
     """
 
-    def __init__(self, proto, inputs, op=ALLREDUCE, first_epoch=1, bug=None):
+    def __init__(self, proto, inputs, op=ALLREDUCE, first_epoch=1, bug=None, sentinel_reset="after_all"):
         x = np.asarray(inputs, dtype=np.uint16)
+        if sentinel_reset not in ("after_all", "on_accept"):
+            raise ValueError(sentinel_reset)
+        # when the sentinel reader writes the fill back: after every source of
+        # the epoch is in ("after_all", the page's order: consume, then reset)
+        # or in the same atomic step that accepts each unit ("on_accept")
+        self.sentinel_reset = sentinel_reset
         if x.ndim != 3:
             raise ValueError("inputs must be [K, N, count]")
         self.proto = proto
@@ -304,6 +310,10 @@ class ChainSim:
                 lo, vals = P.decode_unit(self.proto, slot, j, self.count)
                 rk.staged[q][lo:lo + vals.size] = vals
                 acc[j] = True
+                if self.proto == P.SENTINEL and self.sentinel_reset == "on_accept" and self.bug != "no_reset":
+                    off, body = P.reset_unit_bytes(self.proto, j)
+                    slot[off:off + body.size] = body
+                    self.shadow[(r, par, q)][j] = None
             if acc.all():
                 rk.arrival.append(q)
         if all(rk.accepted[q].all() for q in rk.accepted):
@@ -328,7 +338,7 @@ class ChainSim:
         else:
             self.outputs[k, r] = np.concatenate([rows[q] for q in range(self.N)])
         self.completed[k, r] = True
-        if self.proto == P.SENTINEL and self.bug != "no_reset":
+        if self.proto == P.SENTINEL and self.bug != "no_reset" and self.sentinel_reset == "after_all":
             for q in range(self.N):
                 if q == r:
                     continue
@@ -474,11 +484,11 @@ class ChainSim:
         return v
 
 
-def run_fifo(proto, inputs, op=ALLREDUCE, first_epoch=1):
+def run_fifo(proto, inputs, op=ALLREDUCE, first_epoch=1, sentinel_reset="after_all"):
     """One fixed, cheap schedule for large inputs: in rounds, every rank
     that can push pushes, every pending store lands in issue order, every
     rank polls. Linear in the number of units; returns (sim, violations)."""
-    sim = ChainSim(proto, inputs, op=op, first_epoch=first_epoch)
+    sim = ChainSim(proto, inputs, op=op, first_epoch=first_epoch, sentinel_reset=sentinel_reset)
     while not sim.finished():
         progressed = False
         for r in range(sim.N):
@@ -500,7 +510,7 @@ def run_fifo(proto, inputs, op=ALLREDUCE, first_epoch=1):
 
 
 def run_chain(proto, inputs, op=ALLREDUCE, first_epoch=1, schedule="random", seed=0,
-              slow_rank=None, bug=None, max_steps=2_000_000):
+              slow_rank=None, bug=None, max_steps=2_000_000, sentinel_reset="after_all"):
     """Run one schedule to completion; returns (sim, violations).
 
     ``schedule``: ``"random"`` picks uniformly among enabled actions;
@@ -508,7 +518,7 @@ def run_chain(proto, inputs, op=ALLREDUCE, first_epoch=1, schedule="random", see
     the stores it sent) until nothing else can happen, then lets one through;
     ``"inorder"`` always takes the first enabled action.
     """
-    sim = ChainSim(proto, inputs, op=op, first_epoch=first_epoch, bug=bug)
+    sim = ChainSim(proto, inputs, op=op, first_epoch=first_epoch, bug=bug, sentinel_reset=sentinel_reset)
     rng = np.random.default_rng(seed)
     while not sim.finished() and sim.steps < max_steps:
         acts = sim.enabled_actions()

@@ -135,3 +135,25 @@ def test_fifo_schedule_for_large_inputs(proto):
     x = _x(23, 2, 4, 300)
     _, v = S.run_fifo(proto, x)
     assert not v, v[:3]
+
+
+@pytest.mark.parametrize("n,count,k", [(2, 2, 3), (3, 1, 2)])
+def test_sentinel_reset_on_accept_every_interleaving(n, count, k):
+    """The sentinel variant that writes the fill back in the same atomic step
+    that accepts a unit (no separate reset pass) is as safe as resetting after
+    the whole epoch: every interleaving, no violation."""
+    x = _x(31 + n, k, n, count)
+    states, v = exhaustive.explore_interleavings(P.SENTINEL, x, sentinel_reset="on_accept", max_states=400_000)
+    assert not v, v[:3]
+    _, v = exhaustive.explore_interleavings(P.SENTINEL, x, sentinel_reset="on_accept", bug="no_reset")
+    assert v
+
+
+@pytest.mark.parametrize("n", [2, 4, 8])
+def test_sentinel_reset_on_accept_schedules(n):
+    x = _x(40 + n, 3, n, 13)
+    for seed in range(2):
+        _, v = S.run_chain(P.SENTINEL, x, seed=seed, sentinel_reset="on_accept")
+        assert not v, v[:3]
+    _, v = S.run_chain(P.SENTINEL, x, seed=5, schedule="adversarial", slow_rank=0, sentinel_reset="on_accept")
+    assert not v, v[:3]
