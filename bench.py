@@ -305,9 +305,11 @@ def run_gpu(args):
 
     dom = per_size[-1]  # largest size: most time per step
     ach = dom["achieved_gbs_launch"]
+    key = f"sfc_kernel<{NRANKS}, sentinel, allreduce> x {K_OPS} ops, {dom['bytes_per_rank']} B/rank"
     roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": ach / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks["source"],
-            "kernel": f"sfc_kernel<{NRANKS}, sentinel, allreduce> x {K_OPS} ops, {dom['bytes_per_rank']} B/rank"}
+            "frac": ach / peaks["hbm_gbs"], "traffic": recorded_traffic(key),
+            "algorithmic_bytes_per_launch": dom["algorithmic_bytes_per_op"] * K_OPS,
+            "peak_source": peaks["source"], "kernel": key}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -342,6 +344,35 @@ def run_gpu(args):
     if ws > 1:
         dist.destroy_process_group()
     return 0
+
+
+def kernel_sources_sha():
+    """SHA-256 over the CUDA sources and headers the kernels are built from."""
+    import hashlib
+
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "latency_self_synchronizing_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(name.encode())
+            h.update(open(os.path.join(csrc, name), "rb").read())
+    h.update(open(os.path.join(ROOT, "include", "sfc.h"), "rb").read())
+    return h.hexdigest()
+
+
+def recorded_traffic(key):
+    """DRAM bytes per launch recorded from an ncu capture of this kernel and
+    workload (profiles/ncu_traffic.json), or None when the kernel sources have
+    changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        rec = json.load(open(path))
+    except (OSError, ValueError):
+        return None
+    if rec.get("kernel_sources_sha") != kernel_sources_sha():
+        return None
+    ent = rec.get("launches", {}).get(key)
+    return None if ent is None else float(ent["dram_bytes_per_launch"])
 
 
 def _peaks():
