@@ -92,16 +92,25 @@ typedef struct {
   uint32_t protocol_mask;   /* bit p provisions scratch for protocol p; 0 = all */
 } sfc_config;
 
-/* Latency model of the selector: T = alpha_us + beta_us_per_byte * bytes,
- * bytes = sfc_algorithmic_bytes(op, protocol, count, nranks). An entry with
+/* Latency model of the selector, one entry per (op, protocol, nranks):
+ * table_us[i] is the measured p50 latency (us) at 2^(SFC_COST_MIN_LOG2 + i)
+ * bytes per rank (<= 0: not measured). The estimate at b bytes per rank is the
+ * measured value, interpolated linearly in log2(b) between the nearest
+ * measured sizes, held at the smallest measured value below it, and scaled by
+ * algorithmic bytes (sfc_algorithmic_bytes) above the largest. An entry with
+ * no measured size uses alpha_us + beta_us_per_byte * algorithmic bytes.
  * alpha_us < 0 marks the protocol unavailable for that rank count. */
+#define SFC_COST_BUCKETS 24
+#define SFC_COST_MIN_LOG2 9
+
 typedef struct {
   double alpha_us;
   double beta_us_per_byte;
-} sfc_cost_coeff;
+  double table_us[SFC_COST_BUCKETS];
+} sfc_cost_entry;
 
 typedef struct {
-  sfc_cost_coeff c[2][SFC_NUM_PROTOCOLS][SFC_MAX_RANKS + 1]; /* [op][protocol][nranks] */
+  sfc_cost_entry c[2][SFC_NUM_PROTOCOLS][SFC_MAX_RANKS + 1]; /* [op][protocol][nranks] */
 } sfc_cost_model;
 
 typedef struct {
@@ -182,16 +191,21 @@ sfc_status sfc_allreduce_chain_host(sfc_ctx* ctx, int k_ops, const void* in_host
  * count: "flash-comm: Self-Synchronizing Collective Communication for LLM
  * Decoding", abstract; the empirical choice in "Why Microseconds Matter in AI
  * Infrastructure", section "What I learned from it"). argmin over protocols
- * of alpha + beta * bytes; ties go to fewer bytes, then to the order
- * SENTINEL, LL128, LL, BARRIER_ONESHOT, BARRIER_TWOSHOT. Host only. */
+ * of the model's latency estimate (sfc_cost_estimate); ties go to fewer
+ * algorithmic bytes, then to the order SENTINEL, LL128, LL, BARRIER_ONESHOT,
+ * BARRIER_TWOSHOT. Host only. */
 sfc_protocol sfc_select_protocol(const sfc_ctx* ctx, sfc_op op, size_t bytes_per_rank, int nranks);
 
 /* The same choice from an explicit model; needs no context and no GPU. */
 sfc_protocol sfc_select_protocol_model(const sfc_cost_model* model, sfc_op op,
                                        size_t bytes_per_rank, int nranks);
 
-/* Replace the context's model (copied). The built-in default comes from a
- * fit on B200 measurements. */
+/* The model's latency estimate (us) for one protocol; < 0 if unavailable. */
+double sfc_cost_estimate(const sfc_cost_model* model, sfc_op op, sfc_protocol protocol,
+                         size_t bytes_per_rank, int nranks);
+
+/* Replace the context's model (copied). The built-in default holds p50
+ * latencies measured on a B200 by the message-size sweep. */
 sfc_status sfc_set_cost_model(sfc_ctx* ctx, const sfc_cost_model* model);
 
 /* Write the built-in default model into *model. */

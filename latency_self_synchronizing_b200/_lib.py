@@ -21,12 +21,17 @@ class Config(C.Structure):
                 ("protocol_mask", C.c_uint32)]
 
 
-class CostCoeff(C.Structure):
-    _fields_ = [("alpha_us", C.c_double), ("beta_us_per_byte", C.c_double)]
+SFC_COST_BUCKETS = 24
+SFC_COST_MIN_LOG2 = 9
+
+
+class CostEntry(C.Structure):
+    _fields_ = [("alpha_us", C.c_double), ("beta_us_per_byte", C.c_double),
+                ("table_us", C.c_double * SFC_COST_BUCKETS)]
 
 
 class CostModel(C.Structure):
-    _fields_ = [("c", CostCoeff * (SFC_MAX_RANKS + 1) * SFC_NUM_PROTOCOLS * 2)]
+    _fields_ = [("c", CostEntry * (SFC_MAX_RANKS + 1) * SFC_NUM_PROTOCOLS * 2)]
 
 
 class FloorResult(C.Structure):
@@ -51,6 +56,7 @@ SIGNATURES = [
     ("sfc_select_protocol", C.c_int, [_P, C.c_int, C.c_size_t, C.c_int]),
     ("sfc_select_protocol_model", C.c_int, [C.POINTER(CostModel), C.c_int, C.c_size_t, C.c_int]),
     ("sfc_set_cost_model", _S, [_P, C.POINTER(CostModel)]),
+    ("sfc_cost_estimate", C.c_double, [C.POINTER(CostModel), C.c_int, C.c_int, C.c_size_t, C.c_int]),
     ("sfc_default_cost_model", None, [C.POINTER(CostModel)]),
     ("sfc_algorithmic_bytes", C.c_double, [C.c_int, C.c_int, C.c_size_t, C.c_int]),
     ("sfc_get_status", _S, [_P, C.POINTER(C.c_uint32)]),

@@ -14,7 +14,7 @@ from . import _lib
 
 __all__ = [
     "Status", "Protocol", "Op", "SfcError", "Communicator", "pointer_table", "measure_floor",
-    "algorithmic_bytes", "select_protocol_model", "default_cost_model", "status_string",
+    "algorithmic_bytes", "select_protocol_model", "default_cost_model", "status_string", "cost_estimate",
 ]
 
 
@@ -260,6 +260,11 @@ def default_cost_model():
     m = _lib.CostModel()
     _lib.load().sfc_default_cost_model(C.byref(m))
     return m
+
+
+def cost_estimate(model, op, protocol, bytes_per_rank, nranks):
+    return float(_lib.load().sfc_cost_estimate(C.byref(model), int(as_op(op)), int(as_protocol(protocol)),
+                                               int(bytes_per_rank), int(nranks)))
 
 
 def select_protocol_model(model, op, bytes_per_rank, nranks):

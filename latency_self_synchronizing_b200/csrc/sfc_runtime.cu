@@ -11,6 +11,7 @@
 #include <vector>
 
 #include "sfc.h"
+#include "sfc_cost_table.h"
 #include "sfc_internal.h"
 
 using namespace sfc;
@@ -228,22 +229,18 @@ sfc_status chain(sfc_ctx* c, sfc_op op, int k_ops, const void* const* in_table, 
   return s;
 }
 
-// Built-in latency model. Coefficients per (op, protocol, nranks) were fitted
-// on B200 measurements of the message-size sweep; rank counts that were not
-// measured use the nearest measured one.
+// Built-in latency model: the p50 latencies the message-size sweep measured
+// on a B200 (sfc_cost_table.h); every protocol with a kernel is available.
 void builtin_model(sfc_cost_model* m) {
   std::memset(m, 0, sizeof(*m));
   for (int op = 0; op < 2; ++op)
     for (int pr = 0; pr < SFC_NUM_PROTOCOLS; ++pr)
-      for (int n = 0; n <= SFC_MAX_RANKS; ++n) m->c[op][pr][n] = {-1.0, 0.0};
-  // alpha (us), beta (us per algorithmic byte); placeholders until fitted
-  const double a[6] = {0, 1.5, 2.5, 2.0, 3.0, 4.5};
-  const double b[6] = {0, 1.0 / 5.0e6, 1.0 / 5.0e6, 1.0 / 5.0e6, 1.0 / 5.0e6, 1.0 / 5.0e6};
-  for (int op = 0; op < 2; ++op)
-    for (int pr = 1; pr < SFC_NUM_PROTOCOLS; ++pr)
-      for (int n = kMinRanks; n <= SFC_MAX_RANKS; ++n) {
-        if (op == SFC_OP_ALLGATHER && pr == kTwoshot) continue;
-        m->c[op][pr][n] = {a[pr], b[pr]};
+      for (int n = 0; n <= SFC_MAX_RANKS; ++n) {
+        sfc_cost_entry& e = m->c[op][pr][n];
+        const bool exists = pr >= kLL && n >= kMinRanks && !(op == SFC_OP_ALLGATHER && pr == kTwoshot);
+        e.alpha_us = exists ? 0.0 : -1.0;
+        e.beta_us_per_byte = 0.0;
+        for (int i = 0; i < SFC_COST_BUCKETS; ++i) e.table_us[i] = exists ? kMeasuredP50Us[op][pr][n][i] : -1.0;
       }
 }
 
@@ -296,6 +293,38 @@ void sfc_default_cost_model(sfc_cost_model* model) {
   if (model) builtin_model(model);
 }
 
+double sfc_cost_estimate(const sfc_cost_model* m, sfc_op op, sfc_protocol protocol, size_t bytes_per_rank,
+                         int nranks) {
+  if (m == nullptr || (op != 0 && op != 1) || protocol < SFC_PROTO_LL || protocol > SFC_PROTO_BARRIER_TWOSHOT ||
+      nranks < kMinRanks || nranks > kMaxRanks)
+    return -1.0;
+  const sfc_cost_entry& e = m->c[op][protocol][nranks];
+  if (e.alpha_us < 0) return -1.0;
+  const size_t count = bytes_per_rank / 2;
+  const double bytes = sfc_algorithmic_bytes(op, protocol, count, nranks);
+  if (bytes < 0) return -1.0;
+  int first = -1, last = -1;
+  for (int i = 0; i < SFC_COST_BUCKETS; ++i)
+    if (e.table_us[i] > 0) {
+      if (first < 0) first = i;
+      last = i;
+    }
+  if (first < 0) return e.alpha_us + e.beta_us_per_byte * bytes;
+  const double k = std::log2(static_cast<double>(bytes_per_rank > 0 ? bytes_per_rank : 1)) - SFC_COST_MIN_LOG2;
+  if (k <= first) return e.table_us[first];
+  if (k >= last) {
+    const size_t ref = (static_cast<size_t>(1) << (SFC_COST_MIN_LOG2 + last)) / 2;
+    const double ref_bytes = sfc_algorithmic_bytes(op, protocol, ref, nranks);
+    return e.table_us[last] * (ref_bytes > 0 ? bytes / ref_bytes : 1.0);
+  }
+  int lo = static_cast<int>(std::floor(k));
+  while (lo > first && !(e.table_us[lo] > 0)) --lo;
+  int hi = static_cast<int>(std::ceil(k));
+  while (hi < last && !(e.table_us[hi] > 0)) ++hi;
+  if (hi == lo) return e.table_us[lo];
+  return e.table_us[lo] + (e.table_us[hi] - e.table_us[lo]) * (k - lo) / (hi - lo);
+}
+
 sfc_protocol sfc_select_protocol_model(const sfc_cost_model* m, sfc_op op, size_t bytes_per_rank, int nranks) {
   static const int order[5] = {SFC_PROTO_SENTINEL, SFC_PROTO_LL128, SFC_PROTO_LL, SFC_PROTO_BARRIER_ONESHOT,
                                SFC_PROTO_BARRIER_TWOSHOT};
@@ -305,11 +334,9 @@ sfc_protocol sfc_select_protocol_model(const sfc_cost_model* m, sfc_op op, size_
   double best_t = 0, best_b = 0;
   for (int i = 0; i < 5; ++i) {
     const int pr = order[i];
-    const sfc_cost_coeff cc = m->c[op][pr][nranks];
-    if (cc.alpha_us < 0) continue;
+    const double t = sfc_cost_estimate(m, op, static_cast<sfc_protocol>(pr), bytes_per_rank, nranks);
+    if (t < 0) continue;
     const double b = sfc_algorithmic_bytes(op, static_cast<sfc_protocol>(pr), count, nranks);
-    if (b < 0) continue;
-    const double t = cc.alpha_us + cc.beta_us_per_byte * b;
     if (best == SFC_PROTO_AUTO || t < best_t || (t == best_t && b < best_b)) {
       best = pr;
       best_t = t;

@@ -2,8 +2,8 @@
 
     python -m latency_self_synchronizing_b200.sweep [--nranks 2 4 8] [--op allreduce]
         [--protocols ll ll128 sentinel barrier_oneshot barrier_twoshot]
-        [--min-bytes 1024] [--max-bytes 67108864] [--k-ops 50] [--reps 3]
-        [--out sweep.jsonl] [--fit model.json]
+        [--min-bytes 1024] [--max-bytes 67108864 | --sizes B ...] [--k-ops 50] [--reps 3]
+        [--out sweep.jsonl] [--model-from SWEEP.jsonl ...] [--report selector.json]
 
 For every (rank count, protocol, size) it runs `--reps` chains of `--k-ops`
 operations in one persistent launch each and reports p50 / p99 microseconds
@@ -14,10 +14,12 @@ generator (the sweep checks no values; parity is the tests' job); operations
 cycle through at most 8 distinct inputs per rank so that the largest sizes
 fit.
 
-`--fit` fits, per (op, protocol, N), T = alpha + beta * bytes by least squares
-weighted by 1/T (relative error), and writes the coefficients as JSON; the
-selector's choice under the fitted model is reported at every point together
-with the measured best (regret = chosen p50 / best p50).
+After the sweep the selector is evaluated at every swept size: its choice
+under the latency model (the built-in table, or one built from earlier sweep
+files given with `--model-from`) against the protocol measured fastest there
+(regret = chosen p50 / best p50). `--sizes` sweeps explicit sizes (e.g. the
+midpoints 1.5 * 2^k between the table's measured sizes, for an
+out-of-sample check).
 """
 
 import argparse
@@ -76,35 +78,23 @@ def measure_point(comm, op, proto, count, k_ops, reps, gen, dev):
             "ctas_per_rank": comm.launch_shape(op, proto, count)[0]}
 
 
-def fit(points):
-    """{(op, proto, n): (alpha_us, beta_us_per_byte)} by 1/T-weighted least squares."""
-    groups = {}
+def evaluate_selector(points, model):
+    """Per swept (op, N, size): the model's choice vs the measured fastest."""
+    best = {}
     for p in points:
-        groups.setdefault((p["op"], p["protocol"], p["nranks"]), []).append(p)
-    out = {}
-    for key, pts in groups.items():
-        x = np.array([p["algorithmic_bytes"] for p in pts], dtype=np.float64)
-        y = np.array([p["p50_us"] for p in pts], dtype=np.float64)
-        w = 1.0 / y
-        A = np.stack([np.ones_like(x), x], axis=1) * w[:, None]
-        coef, *_ = np.linalg.lstsq(A, y * w, rcond=None)
-        alpha, beta = float(coef[0]), float(coef[1])
-        if beta < 0:  # flat curve: latency-bound everywhere
-            alpha, beta = float(np.median(y)), 0.0
-        if alpha < 0:
-            alpha = 0.0
-        out[key] = (alpha, beta)
-    return out
-
-
-def model_from_fit(coeffs):
-    m = api.default_cost_model()
-    for (op, proto, n), (a, b) in coeffs.items():
-        o = int(api.as_op(op))
-        pr = int(api.as_protocol(proto))
-        m.c[o][pr][n].alpha_us = a
-        m.c[o][pr][n].beta_us_per_byte = b
-    return m
+        key = (p["op"], p["nranks"], p["bytes_per_rank"])
+        if key not in best or p["p50_us"] < best[key]["p50_us"]:
+            best[key] = p
+    rows = []
+    for key, bp in sorted(best.items()):
+        op, n, nbytes = key
+        chosen = api.select_protocol_model(model, op, nbytes, n).name.lower()
+        cps = [p for p in points if (p["op"], p["nranks"], p["bytes_per_rank"]) == key and p["protocol"] == chosen]
+        if not cps:
+            continue
+        rows.append({"op": op, "nranks": n, "bytes_per_rank": nbytes, "selector": chosen,
+                     "best": bp["protocol"], "regret": cps[0]["p50_us"] / bp["p50_us"]})
+    return rows
 
 
 def main(argv=None):
@@ -118,8 +108,10 @@ def main(argv=None):
     ap.add_argument("--k-ops", type=int, default=50)
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--ctas-per-rank", type=int, default=0)
+    ap.add_argument("--sizes", type=int, nargs="+", default=None, help="explicit bytes per rank")
     ap.add_argument("--out", default=None)
-    ap.add_argument("--fit", default=None)
+    ap.add_argument("--model-from", nargs="+", default=None, help="sweep JSONL files for the selector model")
+    ap.add_argument("--report", default=None, help="write the selector evaluation here (JSON)")
     a = ap.parse_args(argv)
     dev = torch.device("cuda")
     gen = torch.Generator(device=dev)
@@ -129,6 +121,8 @@ def main(argv=None):
     while b <= a.max_bytes:
         sizes.append(b)
         b *= 2
+    if a.sizes:
+        sizes = sorted(a.sizes)
     protos = [p for p in a.protocols if not (a.op == "allgather" and p == "barrier_twoshot")]
     points = []
     sink = open(a.out, "w") if a.out else None
@@ -147,30 +141,23 @@ def main(argv=None):
             finally:
                 comm.close()
                 torch.cuda.empty_cache()
-    if a.fit:
-        coeffs = fit(points)
-        model = model_from_fit(coeffs)
-        best = {}
-        for p in points:
-            key = (p["op"], p["nranks"], p["bytes_per_rank"])
-            if key not in best or p["p50_us"] < best[key]["p50_us"]:
-                best[key] = p
-        regrets = []
-        for key, bp in sorted(best.items()):
-            op, n, nbytes = key
-            chosen = api.select_protocol_model(model, op, nbytes, n).name.lower()
-            cp = next(p for p in points if (p["op"], p["nranks"], p["bytes_per_rank"]) == key
-                      and p["protocol"] == chosen)
-            r = cp["p50_us"] / bp["p50_us"]
-            regrets.append(r)
-            print(json.dumps({"selector": chosen, "best": bp["protocol"], "op": op, "nranks": n,
-                              "bytes_per_rank": nbytes, "regret": r}), flush=True)
-        out = {"coefficients": [{"op": k[0], "protocol": k[1], "nranks": k[2], "alpha_us": v[0],
-                                 "beta_us_per_byte": v[1]} for k, v in sorted(coeffs.items())],
-               "regret_median": statistics.median(regrets), "regret_max": max(regrets)}
-        with open(a.fit, "w") as f:
-            json.dump(out, f, indent=1)
-        print(json.dumps({"regret_median": out["regret_median"], "regret_max": out["regret_max"]}))
+    if a.model_from:
+        from .gen_cost_table import cost_model_from_points, load_points
+
+        model = cost_model_from_points(load_points(a.model_from))
+    else:
+        model = api.default_cost_model()
+    rows = evaluate_selector(points, model)
+    for row in rows:
+        print(json.dumps(dict(row, kind="selector")), flush=True)
+    if rows:
+        regrets = [r["regret"] for r in rows]
+        summary = {"regret_median": statistics.median(regrets), "regret_max": max(regrets),
+                   "points": len(rows)}
+        print(json.dumps(summary), flush=True)
+        if a.report:
+            with open(a.report, "w") as f:
+                json.dump({"summary": summary, "rows": rows}, f, indent=1)
     if sink:
         sink.close()
     return 0

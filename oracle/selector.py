@@ -7,24 +7,27 @@ cost. "Why Microseconds Matter in AI Infrastructure", section "What I learned
 from it": the choice there was made from measurements, a predictive model
 being future work. Neither page gives a functional form or a number.
 
-Reading taken: per protocol p and rank count N a latency estimate
-
-    T_p(S, N) = alpha_p(N) + beta_p(N) * bytes_p(S, N)
-
-where bytes_p is the algorithmic traffic of one operation (encoded bytes
-written plus bytes read over all ranks), alpha and beta are fitted on the
-machine, and the choice is the argmin; on a tie the protocol that moves
-fewer bytes wins, then the earlier one in the order
+Reading taken: per protocol p and rank count N a latency estimate T_p(S, N)
+built from measurements (the empirical selection of the review): the p50
+latency measured at power-of-two message sizes, interpolated linearly in
+log2(S) between the nearest measured sizes, held at the smallest measured
+value below them, and scaled by the algorithmic traffic bytes_p(S, N) above
+the largest; with no measurements, alpha_p(N) + beta_p(N) * bytes_p(S, N)
+(the synchronization cost plus the transfer cost the flash-comm abstract
+weighs). The choice is the argmin; on a tie the protocol that moves fewer
+bytes wins, then the earlier one in the order
 sentinel < LL128 < LL < barrier oneshot < barrier twoshot.
 
 Which protocol wins where cannot be checked against the pages (they give no
-numbers): parity unpinned. The argmin and tie-break are pinned by hand
-examples in the tests.
+numbers): parity unpinned. The estimate and the argmin with its tie-break are
+pinned by hand examples in the tests.
 """
+
+import math
 
 from . import protocols as P
 
-__all__ = ["TIE_ORDER", "algorithmic_bytes", "choose"]
+__all__ = ["TIE_ORDER", "algorithmic_bytes", "estimate", "choose"]
 
 TIE_ORDER = (P.SENTINEL, P.LL128, P.LL, "barrier_oneshot", "barrier_twoshot")
 
@@ -56,19 +59,50 @@ def algorithmic_bytes(proto, count, n, op="allreduce"):
     raise ValueError(proto)
 
 
-def choose(coeffs, count, n, op="allreduce", candidates=None):
-    """argmin over ``coeffs[proto] = (alpha, beta)``; returns the protocol."""
+MIN_LOG2 = 9
+
+
+def estimate(entry, proto, bytes_per_rank, n, op="allreduce"):
+    """Latency estimate of one protocol; ``entry`` = (alpha, beta, table)
+    with table[i] the p50 at 2**(MIN_LOG2 + i) bytes per rank (<= 0 = not
+    measured). None if the protocol is unavailable (alpha < 0)."""
+    alpha, beta, table = entry
+    if alpha < 0:
+        return None
+    b = algorithmic_bytes(proto, bytes_per_rank // 2, n, op)
+    measured = [i for i, t in enumerate(table) if t > 0]
+    if not measured:
+        return alpha + beta * b
+    k = math.log2(max(bytes_per_rank, 1)) - MIN_LOG2
+    first, last = measured[0], measured[-1]
+    if k <= first:
+        return table[first]
+    if k >= last:
+        ref = (2 ** (MIN_LOG2 + last)) // 2
+        return table[last] * b / algorithmic_bytes(proto, ref, n, op)
+    lo = math.floor(k)
+    while lo > first and not table[lo] > 0:
+        lo -= 1
+    hi = math.ceil(k)
+    while hi < last and not table[hi] > 0:
+        hi += 1
+    if hi == lo:
+        return table[lo]
+    return table[lo] + (table[hi] - table[lo]) * (k - lo) / (hi - lo)
+
+
+def choose(model, bytes_per_rank, n, op="allreduce"):
+    """argmin over ``model[proto] = (alpha, beta, table)``; returns the protocol."""
     best = None
     for proto in TIE_ORDER:
-        if proto not in coeffs:
-            continue
-        if candidates is not None and proto not in candidates:
+        if proto not in model:
             continue
         if op == "allgather" and proto == "barrier_twoshot":
             continue
-        alpha, beta = coeffs[proto]
-        b = algorithmic_bytes(proto, count, n, op)
-        t = alpha + beta * b
+        t = estimate(model[proto], proto, bytes_per_rank, n, op)
+        if t is None:
+            continue
+        b = algorithmic_bytes(proto, bytes_per_rank // 2, n, op)
         key = (t, b, TIE_ORDER.index(proto))
         if best is None or key < best[0]:
             best = (key, proto)

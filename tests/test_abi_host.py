@@ -4,6 +4,7 @@ agrees with the oracle's plain restatement. No kernel is launched."""
 import os
 import re
 
+import numpy as np
 import pytest
 
 from latency_self_synchronizing_b200 import _lib, api
@@ -46,35 +47,57 @@ def test_algorithmic_bytes_match_oracle(op, n):
                 osel.algorithmic_bytes(name, count, n, op), rel=1e-12)
 
 
-def _model_from(coeffs):
+def _model_from(entries):
+    """ctypes model from {proto: (alpha, beta, table)}; other protocols off."""
     m = api.default_cost_model()
     for op in range(2):
         for p in range(6):
             for n in range(9):
                 m.c[op][p][n].alpha_us = -1.0
-                m.c[op][p][n].beta_us_per_byte = 0.0
     for op in range(2):
         for p, name in PROTO_NAMES.items():
-            if name in coeffs:
+            if name in entries:
+                a, b, tab = entries[name]
                 for n in range(2, 9):
-                    m.c[op][p][n].alpha_us, m.c[op][p][n].beta_us_per_byte = coeffs[name]
+                    e = m.c[op][p][n]
+                    e.alpha_us, e.beta_us_per_byte = a, b
+                    for i in range(24):
+                        e.table_us[i] = tab[i]
     return m
 
 
-def test_selector_matches_oracle_argmin():
-    coeffs = {"ll": (1.2, 1.0 / 3e6), "ll128": (2.0, 1.0 / 5e6), "sentinel": (2.6, 1.0 / 6e6),
-              "barrier_oneshot": (3.5, 1.0 / 6e6), "barrier_twoshot": (5.0, 1.0 / 6.5e6)}
-    m = _model_from(coeffs)
-    for op in ("allreduce", "allgather"):
-        for n in (2, 4, 8):
-            for b in [1024 << i for i in range(17)]:
-                got = api.select_protocol_model(m, op, b, n)
-                want = osel.choose(coeffs, b // 2, n, op)
-                assert PROTO_NAMES[int(got)] == want, (op, n, b)
+def _random_entries(rng):
+    out = {}
+    for name in PROTO_NAMES.values():
+        tab = [-1.0] * 24
+        for i in sorted(rng.choice(24, size=rng.integers(0, 8), replace=False)):
+            tab[i] = float(rng.uniform(0.5, 500.0))
+        out[name] = (float(rng.uniform(0, 5)), float(rng.uniform(0, 1e-6)), tab)
+    return out
+
+
+def test_cost_estimate_and_selector_match_oracle():
+    rng = np.random.default_rng(0)
+    sizes = [512 << i for i in range(20)] + [3000, 70000, 5_000_000, 1 << 33]
+    for trial in range(20):
+        entries = _random_entries(rng)
+        m = _model_from(entries)
+        for op in ("allreduce", "allgather"):
+            for n in (2, 5, 8):
+                for b in sizes:
+                    for p, name in PROTO_NAMES.items():
+                        if op == "allgather" and name == "barrier_twoshot":
+                            continue
+                        want = osel.estimate(entries[name], name, b, n, op)
+                        got = api.cost_estimate(m, op, p, b, n)
+                        assert got == pytest.approx(want, rel=1e-9), (trial, op, n, b, name)
+                    got = api.select_protocol_model(m, op, b, n)
+                    assert PROTO_NAMES[int(got)] == osel.choose(entries, b, n, op), (trial, op, n, b)
 
 
 def test_selector_ties_prefer_fewer_bytes():
-    m = _model_from({"ll": (1.0, 0.0), "sentinel": (1.0, 0.0)})
+    flat = (0.0, 0.0, [2.0] + [-1.0] * 23)
+    m = _model_from({"ll": flat, "sentinel": flat})
     assert api.select_protocol_model(m, "allreduce", 4096, 4) == api.Protocol.SENTINEL
 
 
@@ -82,7 +105,7 @@ def test_default_model_chooses_a_real_protocol_everywhere():
     m = api.default_cost_model()
     for op in ("allreduce", "allgather"):
         for n in range(2, 9):
-            for b in [1024 << i for i in range(17)]:
+            for b in [512 << i for i in range(20)]:
                 p = api.select_protocol_model(m, op, b, n)
                 assert p != api.Protocol.AUTO
                 if op == "allgather":

@@ -35,26 +35,54 @@ def test_algorithmic_bytes_worked_examples():
     assert selector.algorithmic_bytes("ll128", count, 8) == 8 * (2 * count * 2 + 2 * 7 * 128 * lines)
 
 
+NONE = [-1.0] * 24
+
+
+def _tab(**pts):
+    """table with p50 values at the given log2 sizes, e.g. _tab(b10=2.0)."""
+    t = list(NONE)
+    for k, v in pts.items():
+        t[int(k[1:]) - 9] = v
+    return t
+
+
+def test_estimate_hand_examples():
+    e = (0.0, 0.0, _tab(b10=2.0, b12=4.0, b14=10.0))
+    # below the first measured size: held
+    assert selector.estimate(e, "ll", 512, 4) == 2.0
+    # exactly measured
+    assert selector.estimate(e, "ll", 4096, 4) == 4.0
+    # 2^11 is halfway (in log2) between 2^10 and 2^12: 3.0
+    assert selector.estimate(e, "ll", 2048, 4) == pytest.approx(3.0)
+    # 2^13 halfway between 2^12 (4) and 2^14 (10): 7.0
+    assert selector.estimate(e, "ll", 8192, 4) == pytest.approx(7.0)
+    # above the last: scaled by algorithmic bytes (sentinel-free LL: linear)
+    b16 = selector.algorithmic_bytes("ll", 2 ** 15, 4)
+    b14 = selector.algorithmic_bytes("ll", 2 ** 13, 4)
+    assert selector.estimate(e, "ll", 2 ** 16, 4) == pytest.approx(10.0 * b16 / b14)
+    # no table: alpha + beta * bytes
+    assert selector.estimate((1.5, 1e-6, NONE), "ll", 1024, 4) == pytest.approx(
+        1.5 + 1e-6 * selector.algorithmic_bytes("ll", 512, 4))
+    assert selector.estimate((-1.0, 0.0, NONE), "ll", 1024, 4) is None
+
+
 def test_choose_hand_examples():
-    coeffs = {"ll": (1.0, 1e-3), "sentinel": (3.0, 1e-4), "barrier_oneshot": (5.0, 1e-5)}
-    # 1024 elements, 4 ranks: bytes ll=114688, sentinel=61440*... computed:
-    b_ll = selector.algorithmic_bytes("ll", 1024, 4)
-    b_se = selector.algorithmic_bytes("sentinel", 1024, 4)
-    b_b1 = selector.algorithmic_bytes("barrier_oneshot", 1024, 4)
-    t = {"ll": 1.0 + 1e-3 * b_ll, "sentinel": 3.0 + 1e-4 * b_se, "barrier_oneshot": 5.0 + 1e-5 * b_b1}
-    assert selector.choose(coeffs, 1024, 4) == min(t, key=t.get)
-    # tiny message: the small alpha wins
-    assert selector.choose({"ll": (1.0, 0.0), "sentinel": (2.0, 0.0)}, 8, 2) == "ll"
+    model = {"ll": (0.0, 0.0, _tab(b10=1.0, b20=50.0)),
+             "barrier_twoshot": (0.0, 0.0, _tab(b10=5.0, b20=20.0))}
+    assert selector.choose(model, 1024, 8) == "ll"
+    assert selector.choose(model, 1 << 20, 8) == "barrier_twoshot"
+    # crossing: ll 1 + 49 (k-1)/10, twoshot 5 + 15 (k-1)/10 -> equal at k = 1 + 4/34*10 (~2.18)
+    assert selector.choose(model, 2 ** 11, 8) == "ll"
+    assert selector.choose(model, 2 ** 12, 8) == "barrier_twoshot"
 
 
 def test_choose_tie_breaks_on_bytes_then_order():
+    flat = (0.0, 0.0, _tab(b12=3.0))
     # equal estimates: fewer bytes wins (sentinel moves fewer than LL)
-    assert selector.choose({"ll": (1.0, 0.0), "sentinel": (1.0, 0.0)}, 4096, 4) == "sentinel"
-    # equal estimates and equal bytes cannot happen between distinct layouts
-    # except by construction; the fixed order decides
+    assert selector.choose({"ll": flat, "sentinel": flat}, 4096, 4) == "sentinel"
     assert selector.TIE_ORDER[0] == "sentinel"
 
 
 def test_twoshot_never_chosen_for_allgather():
-    coeffs = {"barrier_twoshot": (0.0, 0.0), "ll": (5.0, 0.0)}
-    assert selector.choose(coeffs, 100, 4, op="allgather") == "ll"
+    model = {"barrier_twoshot": (0.0, 0.0, _tab(b10=0.1)), "ll": (0.0, 0.0, _tab(b10=5.0))}
+    assert selector.choose(model, 1024, 4, op="allgather") == "ll"
