@@ -75,10 +75,20 @@ typedef enum {
   SFC_PROTO_LL128 = 2,
   SFC_PROTO_SENTINEL = 3,
   SFC_PROTO_BARRIER_ONESHOT = 4,  /* pull, top + bottom barrier */
-  SFC_PROTO_BARRIER_TWOSHOT = 5   /* all-reduce only: reduce-scatter + all-gather */
+  SFC_PROTO_BARRIER_TWOSHOT = 5,  /* all-reduce only: reduce-scatter + all-gather */
+  /* pull oneshot with the top barrier only: the caller double-buffers its
+   * inputs (an input passed to operation e is not written again before
+   * operation e + 2 is issued), which takes the place of the bottom barrier
+   * ("SiFAR: Synchronization-Free All-Reduce for Low-Latency LLM Inference",
+   * abstract: dual buffering removes the oneshot bottom barrier) */
+  SFC_PROTO_BARRIER_ONESHOT_DB = 6,
+  /* all-reduce only: reduce-scatter then all-gather, each phase a
+   * self-synchronizing push with LL or sentinel readiness; no barrier */
+  SFC_PROTO_LL_TWOSHOT = 7,
+  SFC_PROTO_SENTINEL_TWOSHOT = 8
 } sfc_protocol;
 
-#define SFC_NUM_PROTOCOLS 6
+#define SFC_NUM_PROTOCOLS 9
 #define SFC_MAX_RANKS 8
 
 typedef enum { SFC_BF16 = 0 } sfc_dtype;
@@ -151,7 +161,7 @@ sfc_status sfc_allreduce(sfc_ctx* ctx, const void* const* in, void* const* out, 
 
 /* One all-gather. in: N device pointers to `count` elements; out: N device
  * pointers to N*count elements; out[r] = in[0] || in[1] || ... || in[N-1].
- * BARRIER_TWOSHOT is not an all-gather algorithm (SFC_ERR_UNSUPPORTED). */
+ * The twoshot protocols are all-reduce algorithms (SFC_ERR_UNSUPPORTED). */
 sfc_status sfc_allgather(sfc_ctx* ctx, const void* const* in, void* const* out, size_t count,
                          sfc_dtype dtype, sfc_protocol protocol, uint32_t epoch, void* stream);
 
@@ -192,8 +202,8 @@ sfc_status sfc_allreduce_chain_host(sfc_ctx* ctx, int k_ops, const void* in_host
  * Decoding", abstract; the empirical choice in "Why Microseconds Matter in AI
  * Infrastructure", section "What I learned from it"). argmin over protocols
  * of the model's latency estimate (sfc_cost_estimate); ties go to fewer
- * algorithmic bytes, then to the order SENTINEL, LL128, LL, BARRIER_ONESHOT,
- * BARRIER_TWOSHOT. Host only. */
+ * algorithmic bytes, then to the order SENTINEL, LL128, LL, SENTINEL_TWOSHOT,
+ * LL_TWOSHOT, BARRIER_ONESHOT_DB, BARRIER_ONESHOT, BARRIER_TWOSHOT. Host only. */
 sfc_protocol sfc_select_protocol(const sfc_ctx* ctx, sfc_op op, size_t bytes_per_rank, int nranks);
 
 /* The same choice from an explicit model; needs no context and no GPU. */
@@ -234,7 +244,9 @@ sfc_status sfc_launch_shape(sfc_ctx* ctx, sfc_op op, sfc_protocol protocol, size
 
 /* Device address and byte size of one receive slot of the scratch, for
  * inspection by tests: rank `rank`'s slot for source `src` (!= rank) at
- * `parity`, under `protocol` (LL, LL128 or SENTINEL). */
+ * `parity` (0 or 1), under a self-synchronizing protocol. For the twoshot
+ * protocols parity 0/1 selects a reduce-scatter slot and 2/3 the all-gather
+ * slot of parity 0/1. */
 sfc_status sfc_scratch_slot(sfc_ctx* ctx, sfc_protocol protocol, int rank, int parity, int src,
                             void** device_ptr, size_t* bytes);
 

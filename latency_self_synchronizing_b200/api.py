@@ -37,6 +37,9 @@ class Protocol(enum.IntEnum):
     SENTINEL = 3
     BARRIER_ONESHOT = 4
     BARRIER_TWOSHOT = 5
+    BARRIER_ONESHOT_DB = 6
+    LL_TWOSHOT = 7
+    SENTINEL_TWOSHOT = 8
 
 
 class Op(enum.IntEnum):
@@ -46,7 +49,9 @@ class Op(enum.IntEnum):
 
 _NAMES = {"auto": Protocol.AUTO, "ll": Protocol.LL, "ll128": Protocol.LL128, "sentinel": Protocol.SENTINEL,
           "barrier_oneshot": Protocol.BARRIER_ONESHOT, "oneshot": Protocol.BARRIER_ONESHOT,
-          "barrier_twoshot": Protocol.BARRIER_TWOSHOT, "twoshot": Protocol.BARRIER_TWOSHOT}
+          "barrier_twoshot": Protocol.BARRIER_TWOSHOT, "twoshot": Protocol.BARRIER_TWOSHOT,
+          "barrier_oneshot_db": Protocol.BARRIER_ONESHOT_DB, "oneshot_db": Protocol.BARRIER_ONESHOT_DB,
+          "ll_twoshot": Protocol.LL_TWOSHOT, "sentinel_twoshot": Protocol.SENTINEL_TWOSHOT}
 
 
 def as_protocol(p):

@@ -11,7 +11,17 @@ constexpr int kMaxRanks = 8;
 constexpr int kMinRanks = 2;
 
 // protocol ids (match sfc_protocol)
-enum : int { kLL = 1, kLL128 = 2, kSentinel = 3, kOneshot = 4, kTwoshot = 5 };
+enum : int {
+  kLL = 1,
+  kLL128 = 2,
+  kSentinel = 3,
+  kOneshot = 4,
+  kTwoshot = 5,
+  kOneshotDB = 6,
+  kLLTwoshot = 7,
+  kSentinelTwoshot = 8,
+  kNumProtocols = 9
+};
 // operations (match sfc_op)
 enum : int { kAllreduce = 0, kAllgather = 1 };
 
@@ -60,7 +70,9 @@ struct KParams {
   uint32_t first_epoch;
 
   uint8_t* scratch;     // protocol region; slot (recv, parity, j) at
-                        // ((recv * 2 + parity) * (N - 1) + j) * slot_stride
+                        // ((recv * 2 + parity) * (N - 1) + j) * slot_stride;
+                        // the twoshot protocols keep their all-gather slots
+                        // after the 2 * N * (N - 1) reduce-scatter slots
   uint64_t slot_stride; // bytes
   uint64_t* bar;        // barrier counters [N][bar_stride]
   int bar_stride;
@@ -78,7 +90,14 @@ struct KParams {
 // Kernel entry for (nranks, protocol, op); null if not provided.
 const void* kernel_for(int nranks, int protocol, int op);
 
-// Encoded slot size (bytes) for `count` elements under the GPU layout.
-uint64_t slot_bytes_gpu(int protocol, uint64_t count);
+// Encoded slot size (bytes) for `count` elements under the GPU layout (the
+// twoshot protocols: for one shard of a `count`-element message).
+uint64_t slot_bytes_gpu(int protocol, uint64_t count, int n);
+
+// Vectors (8 elements) per shard of a `count`-element message over n ranks.
+#ifdef __CUDACC__
+__host__ __device__
+#endif
+inline uint64_t shard_vectors(uint64_t count, int n) { return ((count + 7) / 8 + n - 1) / n; }
 
 }  // namespace sfc

@@ -418,6 +418,179 @@ SFC_DEV bool ll128_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid
   return true;
 }
 
+// ======================================================= self-sync twoshot
+// Reduce-scatter then all-gather, each a self-synchronizing push (LL units or
+// sentinel fill), no barrier. Shards are sv = ceil(nvec / N) vectors; thread
+// position v (0 <= v < sv, the same for every rank) handles vector v of every
+// shard: it pushes vector v of each peer's shard s to rank s, polls and
+// reduces vector v of its own shard, pushes the result to every peer, then
+// polls vector v of every other shard. Each push is control dependent on the
+// polls before it, which orders slot reuse as in the oneshot protocols.
+template <int N, bool kLLenc>
+struct TwoshotSlots {
+  // reduce-scatter slot of `recv` from `src` at `par`, then all-gather slots
+  SFC_DEV static uint8_t* rs(const KParams& p, int recv, int par, int src) { return slot_ptr<N>(p, recv, par, src); }
+  SFC_DEV static uint8_t* ag(const KParams& p, int recv, int par, int src) {
+    return slot_ptr<N>(p, recv, par, src) + static_cast<uint64_t>(2 * N * (N - 1)) * p.slot_stride;
+  }
+};
+
+// Store one 8-element vector into a slot position v, encoded.
+template <bool kLLenc>
+SFC_DEV void push_vec(uint8_t* slot, uint64_t v, uint4 x, uint64_t ehi) {
+  if (kLLenc) {
+    st_rlx_v2u64(slot + ll_off(v, 0), ehi | x.x, ehi | x.y);
+    st_rlx_v2u64(slot + ll_off(v, 1), ehi | x.z, ehi | x.w);
+  } else {
+    st_rlx_v2u64(slot + v * 16, (static_cast<uint64_t>(x.y) << 32) | x.x, (static_cast<uint64_t>(x.w) << 32) | x.z);
+  }
+}
+
+// Poll position v of the slots of the sources in `need` (bit q) until every
+// one is in; the received vectors land in x[q]. Warp-uniform; false = abort.
+template <int N, bool kLLenc>
+SFC_DEV bool poll_vecs(const KParams& p, uint8_t* base, uint64_t v, uint32_t e, uint32_t need, uint4 (&x)[N], int op,
+                       int r) {
+  // slot of source q: base + j(q) * slot_stride, j(q) = q < r ? q : q - 1
+  constexpr uint64_t kFill = ~0ull;
+  // LL: bit q = source q pending; sentinel: bits 2q, 2q+1 = its two units
+  uint32_t pend = 0;
+  if (kLLenc) {
+    pend = need;
+  } else {
+#pragma unroll
+    for (int q = 0; q < N; ++q)
+      if (need & (1u << q)) pend |= 3u << (2 * q);
+  }
+  uint64_t a[N], b[N], c[N], d[N];
+  WarpWait ww;
+  while (true) {
+    const uint32_t cur = pend;
+#pragma unroll
+    for (int q = 0; q < N; ++q) {
+      uint8_t* sq = base + static_cast<uint64_t>(q < r ? q : q - 1) * p.slot_stride;
+      if (kLLenc) {
+        if (cur & (1u << q)) {
+          ld_rlx_v2u64(sq + ll_off(v, 0), a[q], b[q]);
+          ld_rlx_v2u64(sq + ll_off(v, 1), c[q], d[q]);
+        }
+      } else {
+        if (cur & (1u << (2 * q))) a[q] = atom_exch_u64(sq + v * 16, kFill);
+        if (cur & (2u << (2 * q))) b[q] = atom_exch_u64(sq + v * 16 + 8, kFill);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < N; ++q) {
+      if (kLLenc) {
+        if ((cur & (1u << q)) && static_cast<uint32_t>(a[q] >> 32) == e && static_cast<uint32_t>(b[q] >> 32) == e &&
+            static_cast<uint32_t>(c[q] >> 32) == e && static_cast<uint32_t>(d[q] >> 32) == e)
+          pend &= ~(1u << q);
+      } else {
+        if ((cur & (1u << (2 * q))) && a[q] != kFill) pend &= ~(1u << (2 * q));
+        if ((cur & (2u << (2 * q))) && b[q] != kFill) pend &= ~(2u << (2 * q));
+      }
+    }
+    if (!__any_sync(kFull, pend != 0u)) break;
+    if (ww.tick(p, op, r, pend ? __ffs(pend) - 1 : -1)) return false;
+  }
+#pragma unroll
+  for (int q = 0; q < N; ++q) {
+    if (!(need & (1u << q))) continue;
+    if (kLLenc)
+      x[q] = make_uint4(static_cast<uint32_t>(a[q]), static_cast<uint32_t>(b[q]), static_cast<uint32_t>(c[q]),
+                        static_cast<uint32_t>(d[q]));
+    else
+      x[q] = make_uint4(static_cast<uint32_t>(a[q]), static_cast<uint32_t>(a[q] >> 32), static_cast<uint32_t>(b[q]),
+                        static_cast<uint32_t>(b[q] >> 32));
+  }
+  return true;
+}
+
+template <int N, bool kLLenc>
+SFC_DEV bool selfsync_twoshot_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid, uint64_t gstride,
+                                 const Operands& io) {
+  using S = TwoshotSlots<N, kLLenc>;
+  const uint64_t count = p.count;
+  const uint64_t nvec = (count + 7) >> 3;
+  const uint64_t sv = shard_vectors(count, N);
+  const int par = e & 1;
+  const uint64_t ehi = static_cast<uint64_t>(e) << 32;
+  const int lane = threadIdx.x & 31;
+  const uint16_t* in_r = io.in;
+  uint16_t* out_r = io.out;
+  const uint32_t peers = ((1u << N) - 1u) & ~(1u << r);
+
+  // reduce-scatter push: vector v of shard s of my input goes to rank s
+  if (r != p.silent_rank) {
+    for (uint64_t v = gtid; v < sv; v += gstride) {
+#pragma unroll
+      for (int s = 0; s < N; ++s) {
+        if (s == r) continue;
+        const uint64_t vg = s * sv + v;
+        if (vg < nvec) push_vec<kLLenc>(S::rs(p, s, par, r), v, load8(in_r, vg * 8, count), ehi);
+      }
+    }
+  }
+  if (io.in_next != nullptr) {
+    int n = 0;
+    for (uint64_t v = gtid; v < sv && n < 8; v += gstride) {
+#pragma unroll
+      for (int s = 0; s < N; ++s) {
+        const uint64_t vg = s * sv + v;
+        if (vg < nvec && n < 8) {
+          prefetch_l2(io.in_next + vg * 8);
+          ++n;
+        }
+      }
+    }
+  }
+
+  // reduce-scatter poll + reduce, then all-gather push of the result
+  {
+    uint8_t* base = S::rs(p, r, par, r == 0 ? 1 : 0);
+    for (uint64_t vb = gtid - lane; vb < sv; vb += gstride) {
+      const uint64_t v = vb + lane;
+      const uint64_t vg = r * sv + v;
+      const bool act = v < sv && vg < nvec;
+      uint4 x[N];
+      if (!poll_vecs<N, kLLenc>(p, base, v, e, act ? peers : 0u, x, op, r)) return false;
+      if (act) {
+        const uint4 own = load8(in_r, vg * 8, count);
+#pragma unroll
+        for (int q = 0; q < N; ++q)
+          if (q == r) x[q] = own;  // static indices keep x in registers
+        const uint4 y = reduce8<N>(x);
+        store_n(out_r, vg * 8, y, 8, count);
+        if (r != p.silent_rank) {
+#pragma unroll
+          for (int q = 0; q < N; ++q)
+            if (q != r) push_vec<kLLenc>(S::ag(p, q, par, r), v, y, ehi);
+        }
+      }
+    }
+  }
+
+  // all-gather poll: vector v of every other shard
+  {
+    uint8_t* base = S::ag(p, r, par, r == 0 ? 1 : 0);
+    for (uint64_t vb = gtid - lane; vb < sv; vb += gstride) {
+      const uint64_t v = vb + lane;
+      uint32_t need = 0;
+      if (v < sv) {
+#pragma unroll
+        for (int q = 0; q < N; ++q)
+          if (q != r && q * sv + v < nvec) need |= 1u << q;
+      }
+      uint4 x[N];
+      if (!poll_vecs<N, kLLenc>(p, base, v, e, need, x, op, r)) return false;
+#pragma unroll
+      for (int q = 0; q < N; ++q)
+        if (need & (1u << q)) store_n(out_r, (q * sv + v) * 8, x[q], 8, count);
+    }
+  }
+  return true;
+}
+
 // ============================================================ barriers
 // Per-CTA-index barrier: CTA k of rank r publishes (epoch << 2) | phase with
 // a release store and waits until CTA k of every rank has published at least
@@ -443,8 +616,10 @@ SFC_DEV bool cta_barrier(const KParams& p, int r, int k, int op, uint64_t target
 
 // Oneshot (pull): top barrier, read every rank's input, reduce in rank
 // order (all-gather: copy), bottom barrier ("SiFAR: Synchronization-Free
-// All-Reduce for Low-Latency LLM Inference", abstract).
-template <int N, int OP>
+// All-Reduce for Low-Latency LLM Inference", abstract). The dual-buffered
+// variant drops the bottom barrier: the caller alternates two input buffers,
+// which is SiFAR's co-design of communication and model execution.
+template <int N, int OP, bool kDualBuffered>
 SFC_DEV bool oneshot_op(const KParams& p, int r, int k, int op, uint32_t e, uint64_t gtid, uint64_t gstride,
                         const Operands& io) {
   const uint64_t count = p.count;
@@ -467,6 +642,9 @@ SFC_DEV bool oneshot_op(const KParams& p, int r, int k, int op, uint32_t e, uint
       for (int q = 0; q < N; ++q) store_n(out_r, q * count + v * 8, x[q], 8, q * count + count);
     }
   }
+  // with dual-buffered inputs the next operation's top barrier already
+  // orders every reuse of this operation's inputs: no bottom barrier
+  if (kDualBuffered) return true;
   return cta_barrier<N>(p, r, k, op, eb | kPhaseBottom);
 }
 
@@ -515,8 +693,16 @@ SFC_DEV bool twoshot_op(const KParams& p, int r, int k, int op, uint32_t e, uint
 }
 
 // ============================================================== the kernel
+// Two CTAs per SM (at most 128 registers a thread), except the self-sync
+// twoshot kernels for four or more ranks, whose two poll phases keep more
+// sources in flight: one CTA per SM, so they never spill.
+template <int N, int PROTO>
+struct MinBlocks {
+  static constexpr int value = ((PROTO == kLLTwoshot || PROTO == kSentinelTwoshot) && N >= 4) ? 1 : 2;
+};
+
 template <int N, int PROTO, int OP>
-__global__ void __launch_bounds__(kThreads, 2) sfc_kernel(const __grid_constant__ KParams p) {
+__global__ void __launch_bounds__(kThreads, MinBlocks<N, PROTO>::value) sfc_kernel(const __grid_constant__ KParams p) {
   const int r = blockIdx.x / p.G;
   const int k = blockIdx.x - r * p.G;
   const uint64_t gtid = static_cast<uint64_t>(k) * kThreads + threadIdx.x;
@@ -540,7 +726,13 @@ __global__ void __launch_bounds__(kThreads, 2) sfc_kernel(const __grid_constant_
     else if (PROTO == kLL128)
       ok = ll128_op<N, OP>(p, r, op, e, gtid, gstride, io);
     else if (PROTO == kOneshot)
-      ok = oneshot_op<N, OP>(p, r, k, op, e, gtid, gstride, io);
+      ok = oneshot_op<N, OP, false>(p, r, k, op, e, gtid, gstride, io);
+    else if (PROTO == kOneshotDB)
+      ok = oneshot_op<N, OP, true>(p, r, k, op, e, gtid, gstride, io);
+    else if (PROTO == kLLTwoshot)
+      ok = selfsync_twoshot_op<N, true>(p, r, op, e, gtid, gstride, io);
+    else if (PROTO == kSentinelTwoshot)
+      ok = selfsync_twoshot_op<N, false>(p, r, op, e, gtid, gstride, io);
     else
       ok = twoshot_op<N>(p, r, k, op, e, gtid, gstride, io);
     if (!ok) return;
@@ -556,7 +748,7 @@ __global__ void __launch_bounds__(kThreads, 2) sfc_kernel(const __grid_constant_
 namespace {
 template <int N>
 struct Row {
-  static void fill(const void* (&t)[kMaxRanks + 1][6][2]) {
+  static void fill(const void* (&t)[kMaxRanks + 1][kNumProtocols][2]) {
     t[N][kLL][kAllreduce] = reinterpret_cast<const void*>(&sfc_kernel<N, kLL, kAllreduce>);
     t[N][kLL][kAllgather] = reinterpret_cast<const void*>(&sfc_kernel<N, kLL, kAllgather>);
     t[N][kLL128][kAllreduce] = reinterpret_cast<const void*>(&sfc_kernel<N, kLL128, kAllreduce>);
@@ -567,11 +759,17 @@ struct Row {
     t[N][kOneshot][kAllgather] = reinterpret_cast<const void*>(&sfc_kernel<N, kOneshot, kAllgather>);
     t[N][kTwoshot][kAllreduce] = reinterpret_cast<const void*>(&sfc_kernel<N, kTwoshot, kAllreduce>);
     t[N][kTwoshot][kAllgather] = nullptr;
+    t[N][kOneshotDB][kAllreduce] = reinterpret_cast<const void*>(&sfc_kernel<N, kOneshotDB, kAllreduce>);
+    t[N][kOneshotDB][kAllgather] = reinterpret_cast<const void*>(&sfc_kernel<N, kOneshotDB, kAllgather>);
+    t[N][kLLTwoshot][kAllreduce] = reinterpret_cast<const void*>(&sfc_kernel<N, kLLTwoshot, kAllreduce>);
+    t[N][kLLTwoshot][kAllgather] = nullptr;
+    t[N][kSentinelTwoshot][kAllreduce] = reinterpret_cast<const void*>(&sfc_kernel<N, kSentinelTwoshot, kAllreduce>);
+    t[N][kSentinelTwoshot][kAllgather] = nullptr;
   }
 };
 
 struct Table {
-  const void* t[kMaxRanks + 1][6][2] = {};
+  const void* t[kMaxRanks + 1][kNumProtocols][2] = {};
   Table() {
     Row<2>::fill(t);
     Row<3>::fill(t);
@@ -586,12 +784,12 @@ struct Table {
 
 const void* kernel_for(int nranks, int protocol, int op) {
   static const Table table;
-  if (nranks < kMinRanks || nranks > kMaxRanks || protocol < kLL || protocol > kTwoshot || op < 0 || op > 1)
+  if (nranks < kMinRanks || nranks > kMaxRanks || protocol < kLL || protocol >= kNumProtocols || op < 0 || op > 1)
     return nullptr;
   return table.t[nranks][protocol][op];
 }
 
-uint64_t slot_bytes_gpu(int protocol, uint64_t count) {
+uint64_t slot_bytes_gpu(int protocol, uint64_t count, int n) {
   const uint64_t nvec = (count + 7) / 8;
   switch (protocol) {
     case kLL:
@@ -603,6 +801,10 @@ uint64_t slot_bytes_gpu(int protocol, uint64_t count) {
     }
     case kSentinel:
       return nvec * 16;
+    case kLLTwoshot:
+      return ((shard_vectors(count, n) + kLLChunkVecs - 1) / kLLChunkVecs) * kLLChunkBytes;
+    case kSentinelTwoshot:
+      return shard_vectors(count, n) * 16;
     default:
       return 0;
   }

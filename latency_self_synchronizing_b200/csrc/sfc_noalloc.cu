@@ -20,7 +20,7 @@ namespace {
 constexpr int kMaxDevices = 64;
 // Largest message: 4096 bf16 elements (8 KB) per rank, up to 8 ranks. The LL
 // receive slots of both parities for 8 ranks need 2 * 8 * 7 slots of
-// slot_bytes_gpu(LL, 4096) = 16 KB each.
+// slot_bytes_gpu(LL, 4096, n) = 16 KB each.
 constexpr uint64_t kNoAllocSlotBytes = 16384;
 constexpr uint64_t kNoAllocSlots = 2ull * sfc::kMaxRanks * (sfc::kMaxRanks - 1);
 constexpr uint64_t kNoAllocStatusBytes = 256;
@@ -92,7 +92,7 @@ extern "C" sfc_status sfc_allreduce_noalloc(const void* const* in, void* const* 
 
   // Every call starts from a clean slate: LL flags of the previous call
   // (epoch 1 as well) and the status word are cleared on the stream first.
-  const uint64_t slot = slot_bytes_gpu(kLL, count);
+  const uint64_t slot = slot_bytes_gpu(kLL, count, nranks);
   const uint64_t used = 2ull * nranks * (nranks - 1) * slot;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* status = base + kNoAllocSlots * kNoAllocSlotBytes;

@@ -24,9 +24,9 @@ struct sfc_ctx {
   sfc_config cfg{};
   int sm_count = 0;
 
-  uint8_t* region[6] = {};     // per self-sync protocol scratch
-  uint64_t slot_stride[6] = {};
-  uint64_t region_bytes[6] = {};
+  uint8_t* region[kNumProtocols] = {};  // per self-sync protocol scratch
+  uint64_t slot_stride[kNumProtocols] = {};
+  uint64_t region_bytes[kNumProtocols] = {};
   uint64_t* bar = nullptr;
   int bar_stride = 0;
   uint16_t* red = nullptr;
@@ -41,7 +41,7 @@ struct sfc_ctx {
   uint64_t launches = 0;
   sfc_cost_model model{};
 
-  int occupancy[6][2] = {};  // blocks per SM, per (protocol, op), 0 = unknown
+  int occupancy[kNumProtocols][2] = {};  // blocks per SM, per (protocol, op), 0 = unknown
 
   // staging for the host-buffer entry point
   uint16_t* stage_in = nullptr;
@@ -52,6 +52,7 @@ struct sfc_ctx {
 namespace {
 
 constexpr uint32_t kDefaultTimeoutUs = 50000;
+constexpr uint32_t kAllProtocolsMask = ((1u << kNumProtocols) - 1u) & ~1u;
 constexpr int kBarStride = 1024;  // >= any CTAs-per-rank value
 
 bool cuda_ok(cudaError_t e) {
@@ -62,10 +63,13 @@ bool cuda_ok(cudaError_t e) {
   return true;
 }
 
-bool self_sync(int proto) { return proto == kLL || proto == kLL128 || proto == kSentinel; }
+bool self_sync(int proto) {
+  return proto == kLL || proto == kLL128 || proto == kSentinel || proto == kLLTwoshot || proto == kSentinelTwoshot;
+}
+bool twoshot_alg(int proto) { return proto == kTwoshot || proto == kLLTwoshot || proto == kSentinelTwoshot; }
 
 bool provisioned(const sfc_ctx* c, int proto) {
-  const uint32_t mask = c->cfg.protocol_mask ? c->cfg.protocol_mask : 0x3Eu;
+  const uint32_t mask = c->cfg.protocol_mask ? c->cfg.protocol_mask : kAllProtocolsMask;
   return (mask >> proto) & 1u;
 }
 
@@ -103,8 +107,8 @@ int choose_G(sfc_ctx* c, int proto, int op, uint64_t count, int* gmax_out) {
   if (proto == kLL128) {
     const uint64_t lines = (count + kLL128Elems - 1) / kLL128Elems;
     threads_needed = (lines + kLL128LinesPerWarp - 1) / kLL128LinesPerWarp * 32;
-  } else if (proto == kTwoshot) {
-    threads_needed = (nvec + c->nranks - 1) / c->nranks;
+  } else if (twoshot_alg(proto)) {
+    threads_needed = shard_vectors(count, c->nranks);
   } else {
     threads_needed = nvec;
   }
@@ -118,8 +122,8 @@ sfc_status check_common(sfc_ctx* c, sfc_op op, size_t count, sfc_dtype dtype, in
   if (c == nullptr || k_ops < 1) return SFC_ERR_INVALID;
   if (dtype != SFC_BF16) return SFC_ERR_UNSUPPORTED;
   if (op != SFC_OP_ALLREDUCE && op != SFC_OP_ALLGATHER) return SFC_ERR_INVALID;
-  if (proto < kLL || proto > kTwoshot) return SFC_ERR_INVALID;
-  if (op == SFC_OP_ALLGATHER && proto == kTwoshot) return SFC_ERR_UNSUPPORTED;
+  if (proto < kLL || proto >= kNumProtocols) return SFC_ERR_INVALID;
+  if (op == SFC_OP_ALLGATHER && twoshot_alg(proto)) return SFC_ERR_UNSUPPORTED;
   if (!provisioned(c, proto)) return SFC_ERR_UNSUPPORTED;
   if (count > c->max_count) return SFC_ERR_INVALID;
   if (c->poisoned) return SFC_ERR_ABORTED;
@@ -237,10 +241,15 @@ void builtin_model(sfc_cost_model* m) {
     for (int pr = 0; pr < SFC_NUM_PROTOCOLS; ++pr)
       for (int n = 0; n <= SFC_MAX_RANKS; ++n) {
         sfc_cost_entry& e = m->c[op][pr][n];
-        const bool exists = pr >= kLL && n >= kMinRanks && !(op == SFC_OP_ALLGATHER && pr == kTwoshot);
-        e.alpha_us = exists ? 0.0 : -1.0;
+        bool measured = false;
+        for (int i = 0; i < SFC_COST_BUCKETS; ++i) {
+          e.table_us[i] = pr < kCostProtocols ? kMeasuredP50Us[op][pr][n][i] : -1.0;
+          measured = measured || e.table_us[i] > 0;
+        }
+        // a protocol the sweep did not measure is never chosen by default
+        const bool exists = pr >= kLL && n >= kMinRanks && !(op == SFC_OP_ALLGATHER && twoshot_alg(pr));
+        e.alpha_us = exists && measured ? 0.0 : -1.0;
         e.beta_us_per_byte = 0.0;
-        for (int i = 0; i < SFC_COST_BUCKETS; ++i) e.table_us[i] = exists ? kMeasuredP50Us[op][pr][n][i] : -1.0;
       }
 }
 
@@ -265,28 +274,40 @@ const char* sfc_status_string(sfc_status s) {
 }
 
 double sfc_algorithmic_bytes(sfc_op op, sfc_protocol protocol, size_t count, int nranks) {
-  if (nranks < kMinRanks || nranks > kMaxRanks) return -1.0;
+  if (nranks < kMinRanks || nranks > kMaxRanks || (op != 0 && op != 1)) return -1.0;
   const double n = nranks;
   const double s = 2.0 * static_cast<double>(count);
-  double enc;
+  const size_t shard = (count + nranks - 1) / nranks;  // elements per twoshot shard
+  auto ll_enc = [](size_t c) { return 8.0 * static_cast<double>((c + 1) / 2); };
   switch (protocol) {
-    case SFC_PROTO_LL: enc = 8.0 * static_cast<double>((count + 1) / 2); break;
-    case SFC_PROTO_LL128: enc = 128.0 * static_cast<double>((count + kLL128Elems - 1) / kLL128Elems); break;
-    case SFC_PROTO_SENTINEL: enc = s; break;
-    default: enc = 0.0;
+    case SFC_PROTO_LL:
+    case SFC_PROTO_LL128:
+    case SFC_PROTO_SENTINEL: {
+      double enc = s;
+      if (protocol == SFC_PROTO_LL) enc = ll_enc(count);
+      if (protocol == SFC_PROTO_LL128) enc = 128.0 * static_cast<double>((count + kLL128Elems - 1) / kLL128Elems);
+      const double reset = protocol == SFC_PROTO_SENTINEL ? (n - 1) * s : 0.0;
+      const double written = op == SFC_OP_ALLREDUCE ? s : n * s;
+      return n * (s + 2.0 * (n - 1) * enc + written + reset);
+    }
+    case SFC_PROTO_BARRIER_ONESHOT:
+    case SFC_PROTO_BARRIER_ONESHOT_DB:
+      return op == SFC_OP_ALLREDUCE ? n * (n * s + s) : n * (n * s + n * s);
+    case SFC_PROTO_BARRIER_TWOSHOT:
+      return op == SFC_OP_ALLREDUCE ? n * (s + s / n + s + s) : -1.0;
+    case SFC_PROTO_LL_TWOSHOT:
+    case SFC_PROTO_SENTINEL_TWOSHOT: {
+      if (op != SFC_OP_ALLREDUCE) return -1.0;
+      // read own input, push + poll (N-1) encoded shards in each of the two
+      // phases, write the output; the sentinel also rewrites what it consumed
+      const double sh = 2.0 * static_cast<double>(shard);
+      const double enc = protocol == SFC_PROTO_LL_TWOSHOT ? ll_enc(shard) : sh;
+      const double reset = protocol == SFC_PROTO_SENTINEL_TWOSHOT ? 2.0 * (n - 1) * sh : 0.0;
+      return n * (s + 4.0 * (n - 1) * enc + s + reset);
+    }
+    default:
+      return -1.0;
   }
-  if (protocol == SFC_PROTO_LL || protocol == SFC_PROTO_LL128 || protocol == SFC_PROTO_SENTINEL) {
-    const double reset = protocol == SFC_PROTO_SENTINEL ? (n - 1) * s : 0.0;
-    const double written = op == SFC_OP_ALLREDUCE ? s : n * s;
-    return n * (s + 2.0 * (n - 1) * enc + written + reset);
-  }
-  if (protocol == SFC_PROTO_BARRIER_ONESHOT) {
-    return op == SFC_OP_ALLREDUCE ? n * (n * s + s) : n * (n * s + n * s);
-  }
-  if (protocol == SFC_PROTO_BARRIER_TWOSHOT && op == SFC_OP_ALLREDUCE) {
-    return n * (s + s / n + s + s);
-  }
-  return -1.0;
 }
 
 void sfc_default_cost_model(sfc_cost_model* model) {
@@ -295,7 +316,7 @@ void sfc_default_cost_model(sfc_cost_model* model) {
 
 double sfc_cost_estimate(const sfc_cost_model* m, sfc_op op, sfc_protocol protocol, size_t bytes_per_rank,
                          int nranks) {
-  if (m == nullptr || (op != 0 && op != 1) || protocol < SFC_PROTO_LL || protocol > SFC_PROTO_BARRIER_TWOSHOT ||
+  if (m == nullptr || (op != 0 && op != 1) || protocol < SFC_PROTO_LL || protocol >= SFC_NUM_PROTOCOLS ||
       nranks < kMinRanks || nranks > kMaxRanks)
     return -1.0;
   const sfc_cost_entry& e = m->c[op][protocol][nranks];
@@ -326,13 +347,15 @@ double sfc_cost_estimate(const sfc_cost_model* m, sfc_op op, sfc_protocol protoc
 }
 
 sfc_protocol sfc_select_protocol_model(const sfc_cost_model* m, sfc_op op, size_t bytes_per_rank, int nranks) {
-  static const int order[5] = {SFC_PROTO_SENTINEL, SFC_PROTO_LL128, SFC_PROTO_LL, SFC_PROTO_BARRIER_ONESHOT,
-                               SFC_PROTO_BARRIER_TWOSHOT};
+  static const int order[8] = {SFC_PROTO_SENTINEL,         SFC_PROTO_LL128,
+                               SFC_PROTO_LL,               SFC_PROTO_SENTINEL_TWOSHOT,
+                               SFC_PROTO_LL_TWOSHOT,       SFC_PROTO_BARRIER_ONESHOT_DB,
+                               SFC_PROTO_BARRIER_ONESHOT,  SFC_PROTO_BARRIER_TWOSHOT};
   if (m == nullptr || nranks < kMinRanks || nranks > kMaxRanks || (op != 0 && op != 1)) return SFC_PROTO_AUTO;
   const size_t count = bytes_per_rank / 2;
   int best = SFC_PROTO_AUTO;
   double best_t = 0, best_b = 0;
-  for (int i = 0; i < 5; ++i) {
+  for (int i = 0; i < 8; ++i) {
     const int pr = order[i];
     const double t = sfc_cost_estimate(m, op, static_cast<sfc_protocol>(pr), bytes_per_rank, nranks);
     if (t < 0) continue;
@@ -368,7 +391,7 @@ sfc_status sfc_init(sfc_ctx** out, int nranks, size_t max_bytes_per_rank, const 
   *out = nullptr;
   if (nranks < kMinRanks || nranks > kMaxRanks || max_bytes_per_rank == 0) return SFC_ERR_INVALID;
   if (cfg && (cfg->ctas_per_rank < 0 || cfg->ctas_per_rank > kBarStride)) return SFC_ERR_INVALID;
-  if (cfg && (cfg->protocol_mask & ~0x3Eu)) return SFC_ERR_INVALID;
+  if (cfg && (cfg->protocol_mask & ~kAllProtocolsMask)) return SFC_ERR_INVALID;
   sfc_ctx* c = new sfc_ctx();
   if (cfg) c->cfg = *cfg;
   c->nranks = nranks;
@@ -386,11 +409,12 @@ sfc_status sfc_init(sfc_ctx** out, int nranks, size_t max_bytes_per_rank, const 
   if (!cuda_ok(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, c->device)) || !coop)
     return fail(SFC_ERR_UNSUPPORTED);
   const uint64_t slots = static_cast<uint64_t>(nranks) * 2 * (nranks - 1);
-  for (int pr : {kLL, kLL128, kSentinel}) {
+  for (int pr : {kLL, kLL128, kSentinel, kLLTwoshot, kSentinelTwoshot}) {
     if (!provisioned(c, pr)) continue;
-    const uint64_t sb = (slot_bytes_gpu(pr, c->max_count) + 255) / 256 * 256;
+    const uint64_t sb = (slot_bytes_gpu(pr, c->max_count, nranks) + 255) / 256 * 256;
     c->slot_stride[pr] = sb;
-    c->region_bytes[pr] = sb * slots;
+    // twoshot: reduce-scatter slots, then as many all-gather slots
+    c->region_bytes[pr] = sb * slots * (pr == kLLTwoshot || pr == kSentinelTwoshot ? 2 : 1);
     if (!cuda_ok(cudaMalloc(&c->region[pr], c->region_bytes[pr]))) return fail(SFC_ERR_CUDA);
   }
   c->bar_stride = kBarStride;
@@ -429,9 +453,9 @@ sfc_status sfc_destroy(sfc_ctx* c) {
 sfc_status sfc_reset(sfc_ctx* c, void* stream) {
   if (c == nullptr) return SFC_ERR_INVALID;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  for (int pr : {kLL, kLL128, kSentinel}) {
+  for (int pr : {kLL, kLL128, kSentinel, kLLTwoshot, kSentinelTwoshot}) {
     if (c->region[pr] == nullptr) continue;
-    const int fill = pr == kSentinel ? 0xFF : 0x00;
+    const int fill = (pr == kSentinel || pr == kSentinelTwoshot) ? 0xFF : 0x00;
     if (!cuda_ok(cudaMemsetAsync(c->region[pr], fill, c->region_bytes[pr], st))) return SFC_ERR_CUDA;
   }
   if (!cuda_ok(cudaMemsetAsync(c->bar, 0, sizeof(uint64_t) * c->nranks * c->bar_stride, st))) return SFC_ERR_CUDA;
@@ -532,7 +556,7 @@ sfc_status sfc_launch_shape(sfc_ctx* c, sfc_op op, sfc_protocol protocol, size_t
   if (c == nullptr || (op != 0 && op != 1)) return SFC_ERR_INVALID;
   int proto = protocol;
   if (proto == SFC_PROTO_AUTO) proto = sfc_select_protocol(c, op, count * 2, c->nranks);
-  if (proto < kLL || proto > kTwoshot) return SFC_ERR_INVALID;
+  if (proto < kLL || proto >= kNumProtocols) return SFC_ERR_INVALID;
   if (kernel_for(c->nranks, proto, op) == nullptr) return SFC_ERR_UNSUPPORTED;
   const int G = choose_G(c, proto, op, count, nullptr);
   if (G <= 0) return SFC_ERR_RESOURCES;
@@ -546,10 +570,13 @@ sfc_status sfc_scratch_slot(sfc_ctx* c, sfc_protocol protocol, int rank, int par
   if (c == nullptr || ptr == nullptr) return SFC_ERR_INVALID;
   const int pr = protocol;
   if (!self_sync(pr) || c->region[pr] == nullptr) return SFC_ERR_UNSUPPORTED;
-  if (rank < 0 || rank >= c->nranks || src < 0 || src >= c->nranks || src == rank || (parity != 0 && parity != 1))
+  const bool two = pr == kLLTwoshot || pr == kSentinelTwoshot;
+  if (rank < 0 || rank >= c->nranks || src < 0 || src >= c->nranks || src == rank || parity < 0 ||
+      parity > (two ? 3 : 1))
     return SFC_ERR_INVALID;
   const int j = src < rank ? src : src - 1;
-  const uint64_t idx = static_cast<uint64_t>((rank * 2 + parity) * (c->nranks - 1) + j);
+  uint64_t idx = static_cast<uint64_t>((rank * 2 + (parity & 1)) * (c->nranks - 1) + j);
+  if (parity >= 2) idx += static_cast<uint64_t>(2 * c->nranks * (c->nranks - 1));  // all-gather slots
   *ptr = c->region[pr] + idx * c->slot_stride[pr];
   if (bytes) *bytes = c->slot_stride[pr];
   return SFC_OK;

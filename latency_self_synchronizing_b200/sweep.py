@@ -102,7 +102,8 @@ def main(argv=None):
     ap.add_argument("--nranks", type=int, nargs="+", default=[2, 4, 8])
     ap.add_argument("--op", default="allreduce", choices=["allreduce", "allgather"])
     ap.add_argument("--protocols", nargs="+",
-                    default=["ll", "ll128", "sentinel", "barrier_oneshot", "barrier_twoshot"])
+                    default=["ll", "ll128", "sentinel", "barrier_oneshot", "barrier_twoshot", "barrier_oneshot_db",
+                             "ll_twoshot", "sentinel_twoshot"])
     ap.add_argument("--min-bytes", type=int, default=1024)
     ap.add_argument("--max-bytes", type=int, default=64 << 20)
     ap.add_argument("--k-ops", type=int, default=50)
@@ -123,7 +124,8 @@ def main(argv=None):
         b *= 2
     if a.sizes:
         sizes = sorted(a.sizes)
-    protos = [p for p in a.protocols if not (a.op == "allgather" and p == "barrier_twoshot")]
+    ar_only = ("barrier_twoshot", "ll_twoshot", "sentinel_twoshot")
+    protos = [p for p in a.protocols if not (a.op == "allgather" and p in ar_only)]
     points = []
     sink = open(a.out, "w") if a.out else None
     for n in a.nranks:

@@ -29,7 +29,7 @@ import numpy as np
 from . import protocols as P
 from . import reference
 from .bf16 import bf16_bits_to_f32, f32_to_bf16_bits
-from .simulator import ChainSim
+from .simulator import _make_sim
 
 __all__ = ["landing_subsets", "arrival_orders", "explore_interleavings"]
 
@@ -137,9 +137,9 @@ def arrival_orders(inputs, bug=None):
 
 
 def explore_interleavings(proto, inputs, op="allreduce", bug=None, max_states=2_000_000,
-                          sentinel_reset="after_all"):
+                          sentinel_reset="after_all", vector=8):
     """Depth-first search over all interleavings; returns (states, violations)."""
-    root = ChainSim(proto, inputs, op=op, bug=bug, sentinel_reset=sentinel_reset)
+    root = _make_sim(proto, inputs, op, 1, bug, sentinel_reset, vector)
     seen = set()
     stack = [root]
     violations = []

@@ -29,7 +29,8 @@ from . import protocols as P
 
 __all__ = ["TIE_ORDER", "algorithmic_bytes", "estimate", "choose"]
 
-TIE_ORDER = (P.SENTINEL, P.LL128, P.LL, "barrier_oneshot", "barrier_twoshot")
+TIE_ORDER = (P.SENTINEL, P.LL128, P.LL, "sentinel_twoshot", "ll_twoshot", "barrier_oneshot_db",
+             "barrier_oneshot", "barrier_twoshot")
 
 
 def algorithmic_bytes(proto, count, n, op="allreduce"):
@@ -50,12 +51,20 @@ def algorithmic_bytes(proto, count, n, op="allreduce"):
         if op == "allreduce":
             return n * (s + 2 * (n - 1) * enc + s + reset)
         return n * (s + 2 * (n - 1) * enc + n * s + reset)
-    if proto == "barrier_oneshot":
+    if proto in ("barrier_oneshot", "barrier_oneshot_db"):
         if op == "allreduce":
             return n * (n * s + s)
         return n * (n * s + n * s)
     if proto == "barrier_twoshot":
         return n * (s + s / n + s + s)
+    if proto in ("ll_twoshot", "sentinel_twoshot"):
+        # read own input, push and poll N-1 encoded shards in each of the two
+        # phases, write the output; the sentinel rewrites what it consumed
+        shard = -(-count // n)
+        sh = 2 * shard
+        enc = P.slot_bytes(P.LL, shard) if proto == "ll_twoshot" else sh
+        reset = 2 * (n - 1) * sh if proto == "sentinel_twoshot" else 0
+        return n * (s + 4 * (n - 1) * enc + s + reset)
     raise ValueError(proto)
 
 
@@ -97,7 +106,7 @@ def choose(model, bytes_per_rank, n, op="allreduce"):
     for proto in TIE_ORDER:
         if proto not in model:
             continue
-        if op == "allgather" and proto == "barrier_twoshot":
+        if op == "allgather" and proto in ("barrier_twoshot", "ll_twoshot", "sentinel_twoshot"):
             continue
         t = estimate(model[proto], proto, bytes_per_rank, n, op)
         if t is None:

@@ -66,11 +66,16 @@ from . import protocols as P
 from . import reference
 from .bf16 import BF16_SENTINEL, bf16_bits_to_f32, f32_to_bf16_bits
 
-__all__ = ["ChainSim", "run_chain", "run_fifo", "BARRIER_ONESHOT", "BARRIER_TWOSHOT", "ALL_PROTOCOLS"]
+__all__ = ["ChainSim", "run_chain", "run_fifo", "BARRIER_ONESHOT", "BARRIER_TWOSHOT", "BARRIER_ONESHOT_DB",
+           "ALL_PROTOCOLS"]
 
 BARRIER_ONESHOT = "barrier_oneshot"
 BARRIER_TWOSHOT = "barrier_twoshot"
-ALL_PROTOCOLS = P.SELF_SYNC + (BARRIER_ONESHOT, BARRIER_TWOSHOT)
+# SiFAR's oneshot with dual-buffered inputs: the caller alternates two input
+# buffers per rank (operation k writes buffer k % 2), so no bottom barrier
+BARRIER_ONESHOT_DB = "barrier_oneshot_db"
+BARRIER_PROTOCOLS = (BARRIER_ONESHOT, BARRIER_TWOSHOT, BARRIER_ONESHOT_DB)
+ALL_PROTOCOLS = P.SELF_SYNC + BARRIER_PROTOCOLS
 
 ALLREDUCE = "allreduce"
 ALLGATHER = "allgather"
@@ -126,7 +131,7 @@ class ChainSim:
         self.pending = []  # list of store records (dicts)
         if proto in P.SELF_SYNC:
             self._init_self_sync()
-        elif proto in (BARRIER_ONESHOT, BARRIER_TWOSHOT):
+        elif proto in BARRIER_PROTOCOLS:
             if proto == BARRIER_TWOSHOT and op != ALLREDUCE:
                 raise ValueError("twoshot is an all-reduce algorithm")
             self._init_barrier()
@@ -156,7 +161,7 @@ class ChainSim:
         self.bar = [0] * self.N
         # input buffer of each rank: (op index it holds, data); the producer
         # of operation k writes it when the rank starts operation k.
-        self.inbuf = [(-1, np.zeros(self.count, dtype=np.uint16)) for _ in range(self.N)]
+        self.inbuf = [[(-1, np.zeros(self.count, dtype=np.uint16)) for _ in range(2)] for _ in range(self.N)]
         shard = -(-self.count // self.N)
         self.shard = shard
         self.redbuf = [(-1, np.zeros(shard, dtype=np.uint16)) for _ in range(self.N)]
@@ -233,7 +238,7 @@ class ChainSim:
             for rk in self.ranks:
                 parts.append((rk.op, rk.phase, tuple(sorted(rk.pulled))))
             parts.append(tuple(self.bar))
-            parts.append(tuple(b[0] for b in self.inbuf))
+            parts.append(tuple(b[0] for bufs in self.inbuf for b in bufs))
             parts.append(tuple(b[0] for b in self.redbuf))
         pend = sorted((s["dst"], s["par"], s["src"], s["j"], s["epoch"]) for s in self.pending)
         parts.append(tuple(pend))
@@ -373,7 +378,7 @@ class ChainSim:
         ph = rk.phase
         if ph == "produce":
             # the producer of operation k overwrites this rank's input buffer
-            self.inbuf[r] = (k, self.inputs[k, r].copy())
+            self.inbuf[r][self._inslot(k)] = (k, self.inputs[k, r].copy())
             rk.pulled = {}
             rk.phase = "arrive_top"
         elif ph == "arrive_top":
@@ -382,9 +387,9 @@ class ChainSim:
         elif ph == "wait_top":
             rk.phase = "pull"
         elif ph == "pull":
-            if self.proto == BARRIER_ONESHOT:
+            if self.proto in (BARRIER_ONESHOT, BARRIER_ONESHOT_DB):
                 src = next(q for q in range(N) if q not in rk.pulled)
-                tag, data = self.inbuf[src]
+                tag, data = self.inbuf[src][self._inslot(k)]
                 if tag != k:
                     self.violations.append(
                         f"rank {r} op {k} pulled rank {src}'s input holding op {tag}")
@@ -396,10 +401,10 @@ class ChainSim:
                     else:
                         self.outputs[k, r] = rows.reshape(-1)
                     self.completed[k, r] = True
-                    rk.phase = "arrive_bottom"
+                    rk.phase = "next" if self.proto == BARRIER_ONESHOT_DB else "arrive_bottom"
             else:  # twoshot reduce-scatter: shard r of every input
                 src = next(q for q in range(N) if q not in rk.pulled)
-                tag, data = self.inbuf[src]
+                tag, data = self.inbuf[src][self._inslot(k)]
                 if tag != k:
                     self.violations.append(
                         f"rank {r} op {k} pulled rank {src}'s input holding op {tag}")
@@ -441,6 +446,12 @@ class ChainSim:
             rk.op += 1
             rk.pulled = {}
             rk.phase = "produce" if rk.op < self.K else "done"
+
+    def _inslot(self, k):
+        """Input buffer that operation k uses: alternating under dual buffering."""
+        if self.proto == BARRIER_ONESHOT_DB and self.bug != "single_input_buffer":
+            return k % 2
+        return 0
 
     def _shard_range(self, q):
         lo = min(q * self.shard, self.count)
@@ -485,26 +496,18 @@ class ChainSim:
 
 
 def run_fifo(proto, inputs, op=ALLREDUCE, first_epoch=1, sentinel_reset="after_all"):
-    """One fixed, cheap schedule for large inputs: in rounds, every rank
-    that can push pushes, every pending store lands in issue order, every
-    rank polls. Linear in the number of units; returns (sim, violations)."""
-    sim = ChainSim(proto, inputs, op=op, first_epoch=first_epoch, sentinel_reset=sentinel_reset)
+    """One fixed, cheap schedule for large inputs: in rounds, every rank takes
+    its enabled step, then every pending store lands in issue order.
+    Linear in the number of units; returns (sim, violations)."""
+    sim = _make_sim(proto, inputs, op, first_epoch, None, sentinel_reset)
     while not sim.finished():
-        progressed = False
-        for r in range(sim.N):
-            if sim.ranks[r].phase != "done" and (proto not in P.SELF_SYNC or sim.ranks[r].phase == "push"):
-                if proto in P.SELF_SYNC or sim._barrier_can_step(r):
-                    sim.apply(("step", r))
-                    progressed = True
+        steps = [a for a in sim.enabled_actions() if a[0] == "step"]
+        for a in steps:
+            sim.apply(a)
+        landed = bool(sim.pending)
         while sim.pending:
             sim.apply(("land", 0))
-            progressed = True
-        if proto in P.SELF_SYNC:
-            for r in range(sim.N):
-                if sim.ranks[r].phase == "poll" and sim._poll_would_progress(r):
-                    sim.apply(("step", r))
-                    progressed = True
-        if not progressed:
+        if not steps and not landed:
             break
     return sim, sim.final_checks()
 
@@ -518,7 +521,7 @@ def run_chain(proto, inputs, op=ALLREDUCE, first_epoch=1, schedule="random", see
     the stores it sent) until nothing else can happen, then lets one through;
     ``"inorder"`` always takes the first enabled action.
     """
-    sim = ChainSim(proto, inputs, op=op, first_epoch=first_epoch, bug=bug, sentinel_reset=sentinel_reset)
+    sim = _make_sim(proto, inputs, op, first_epoch, bug, sentinel_reset)
     rng = np.random.default_rng(seed)
     while not sim.finished() and sim.steps < max_steps:
         acts = sim.enabled_actions()
@@ -530,7 +533,8 @@ def run_chain(proto, inputs, op=ALLREDUCE, first_epoch=1, schedule="random", see
             def is_slow(a):
                 if a[0] == "step":
                     return a[1] == slow_rank
-                return sim.pending[a[1]]["src"] == slow_rank
+                st = sim.pending[a[1]]
+                return (st["src"] if "src" in st else st["key"][3]) == slow_rank
 
             fast = [a for a in acts if not is_slow(a)]
             pool = fast if fast else acts
@@ -539,3 +543,263 @@ def run_chain(proto, inputs, op=ALLREDUCE, first_epoch=1, schedule="random", see
             act = acts[rng.integers(len(acts))]
         sim.apply(act)
     return sim, sim.final_checks()
+
+
+# --------------------------------------------------------------------------
+# Self-synchronizing twoshot: reduce-scatter then all-gather, each phase a
+# self-synchronizing push with the same readiness encodings and epoch-parity
+# double buffering; no barrier anywhere. The large-message variant of the
+# same path (twoshot moves 2(N-1)/N of a message per rank instead of N-1
+# copies; "SiFAR: Synchronization-Free All-Reduce for Low-Latency LLM
+# Inference", abstract: twoshot does better at higher TP degrees).
+LL_TWOSHOT = "ll_twoshot"
+SENTINEL_TWOSHOT = "sentinel_twoshot"
+SELF_SYNC_TWOSHOT = (LL_TWOSHOT, SENTINEL_TWOSHOT)
+ALL_PROTOCOLS = ALL_PROTOCOLS + SELF_SYNC_TWOSHOT
+__all__ += ["TwoshotSim", "LL_TWOSHOT", "SENTINEL_TWOSHOT", "SELF_SYNC_TWOSHOT", "shard_bounds"]
+
+
+def shard_bounds(count, n, q, vector=8):
+    """Elements [lo, hi) of shard q: shards are whole `vector`-element
+    vectors, ceil(ceil(count / vector) / n) of them each; the last ones may be
+    short or empty. (The partition changes no result; tiny exhaustive checks
+    use vector=1 so that every shard holds data.)"""
+    sz = vector * (-(-(-(-count // vector)) // n))
+    lo = min(q * sz, count)
+    return lo, min(lo + sz, count)
+
+
+class TwoshotSim:
+    """K chained self-synchronizing twoshot all-reduces on N ranks.
+
+    Observation from this model: each slot of either phase is written again
+    only after a full exchange of the other phase, so even a single buffer
+    (no parity) passes every check here; the GPU keeps the epoch-parity
+    double buffer of the oneshot protocols all the same.
+
+    Per operation at epoch e, rank r: (1) pushes shard s of its input into
+    rank s's reduce-scatter slot (parity e & 1, source r) for every s != r;
+    (2) polls its reduce-scatter slots until shard r of every peer's input is
+    in, and reduces shard r in rank order (own part from its input); (3)
+    pushes the reduced shard into every peer's all-gather slot; (4) polls its
+    all-gather slots until every other shard is in; the output is the shards
+    in order. Same unit atomicity, shadow tags and checks as ``ChainSim``.
+    """
+
+    def __init__(self, proto, inputs, first_epoch=1, bug=None, sentinel_reset="after_all", vector=8):
+        if proto not in SELF_SYNC_TWOSHOT:
+            raise ValueError(proto)
+        x = np.asarray(inputs, dtype=np.uint16)
+        self.proto = proto
+        self.enc = P.LL if proto == LL_TWOSHOT else P.SENTINEL
+        self.inputs = x
+        self.K, self.N, self.count = x.shape
+        self.first_epoch = first_epoch
+        self.bug = bug
+        self.sentinel_reset = sentinel_reset
+        self.violations = []
+        self.steps = 0
+        self.outputs = np.zeros((self.K, self.N, self.count), dtype=np.uint16)
+        self.pending = []
+        self.bounds = [shard_bounds(self.count, self.N, q, vector) for q in range(self.N)]
+        self.mem, self.shadow = {}, {}
+        for r in range(self.N):
+            for par in (0, 1):
+                for q in range(self.N):
+                    if q == r:
+                        continue
+                    # reduce-scatter slot carries shard r; all-gather slot shard q
+                    for region, sh in (("rs", r), ("ag", q)):
+                        n_el = self.bounds[sh][1] - self.bounds[sh][0]
+                        key = (region, r, par, q)
+                        self.mem[key] = P.initial_slot(self.enc, n_el)
+                        self.shadow[key] = [None] * P.unit_count(self.enc, n_el)
+        # consumed[region] = last epoch whose slots of that region the rank
+        # has fully read
+        self.ranks = [dict(op=0, phase="rs_push", acc={}, staged={}, red=None, consumed={"rs": 0, "ag": 0})
+                      for _ in range(self.N)]
+        for r in range(self.N):
+            self._begin(r)
+
+    def _epoch(self, k):
+        return self.first_epoch + k
+
+    def _par(self, e):
+        return 0 if self.bug == "single_buffer" else e & 1
+
+    def _n_el(self, region, recv, src):
+        sh = recv if region == "rs" else src
+        return self.bounds[sh][1] - self.bounds[sh][0]
+
+    def _begin(self, r):
+        rk = self.ranks[r]
+        rk["acc"], rk["staged"] = {}, {}
+        for region in ("rs", "ag"):
+            for q in range(self.N):
+                if q != r:
+                    n_el = self._n_el(region, r, q)
+                    rk["acc"][(region, q)] = np.zeros(P.unit_count(self.enc, n_el), dtype=bool)
+                    rk["staged"][(region, q)] = np.zeros(n_el, dtype=np.uint16)
+        rk["phase"] = "rs_push" if rk["op"] < self.K else "done"
+
+    # interface ------------------------------------------------------------
+    def finished(self):
+        return all(rk["phase"] == "done" for rk in self.ranks)
+
+    def enabled_actions(self):
+        acts = []
+        for r, rk in enumerate(self.ranks):
+            ph = rk["phase"]
+            if ph in ("rs_push", "ag_push") or (ph in ("rs_poll", "ag_poll") and self._productive(r)):
+                acts.append(("step", r))
+        acts.extend(("land", i) for i in range(len(self.pending)))
+        return acts
+
+    def apply(self, act):
+        self.steps += 1
+        kind, arg = act
+        if kind == "land":
+            self._land(self.pending.pop(arg))
+            return
+        rk = self.ranks[arg]
+        if rk["phase"] == "rs_push":
+            self._push(arg, "rs")
+            rk["phase"] = "rs_poll"
+        elif rk["phase"] == "ag_push":
+            self._push(arg, "ag")
+            rk["phase"] = "ag_poll"
+        else:
+            self._poll(arg, rk["phase"][:2])
+
+    def clone(self):
+        return copy.deepcopy(self)
+
+    def state_key(self):
+        parts = []
+        for key in sorted(self.mem):
+            parts.append(self.mem[key].tobytes())
+            parts.append(tuple(self.shadow[key]))
+        for rk in self.ranks:
+            acc = tuple(rk["acc"][k].tobytes() for k in sorted(rk["acc"]))
+            stg = tuple(rk["staged"][k].tobytes() for k in sorted(rk["staged"]))
+            red = None if rk["red"] is None else rk["red"].tobytes()
+            parts.append((rk["op"], rk["phase"], acc, stg, red))
+        parts.append(tuple(sorted((s["key"], s["j"], s["epoch"]) for s in self.pending)))
+        return tuple(parts)
+
+    # steps ----------------------------------------------------------------
+    def _push(self, r, region):
+        rk = self.ranks[r]
+        k = rk["op"]
+        e = self._epoch(k)
+        par = self._par(e)
+        for p in range(self.N):
+            if p == r:
+                continue
+            if region == "rs":
+                lo, hi = self.bounds[p]
+                data = self.inputs[k, r, lo:hi]
+            else:
+                data = rk["red"]
+            for j, (off, body) in enumerate(P.encode_all(self.enc, data, e)):
+                self.pending.append(dict(key=(region, p, par, r), j=j, off=off, body=body, epoch=e))
+
+    def _land(self, s):
+        key = s["key"]
+        prev = self.shadow[key][s["j"]]
+        reader = self.ranks[key[1]]
+        if prev is not None and prev[1] != s["epoch"] and reader["consumed"][key[0]] < prev[1]:
+            self.violations.append(f"store of epoch {s['epoch']} overwrote unconsumed epoch {prev[1]} in {key}")
+        buf = self.mem[key]
+        buf[s["off"]:s["off"] + s["body"].size] = s["body"]
+        self.shadow[key][s["j"]] = (key[3], s["epoch"])
+
+    def _productive(self, r):
+        rk = self.ranks[r]
+        region = rk["phase"][:2]
+        e = self._epoch(rk["op"])
+        par = self._par(e)
+        for (reg, q), acc in rk["acc"].items():
+            if reg != region:
+                continue
+            slot = self.mem[(region, r, par, q)]
+            for j in range(acc.size):
+                if not acc[j] and P.validate_unit(self.enc, slot, j, e):
+                    return True
+        return all(acc.all() for (reg, _), acc in rk["acc"].items() if reg == region)
+
+    def _poll(self, r, region):
+        rk = self.ranks[r]
+        k = rk["op"]
+        e = self._epoch(k)
+        par = self._par(e)
+        for (reg, q), acc in rk["acc"].items():
+            if reg != region or acc.all():
+                continue
+            key = (region, r, par, q)
+            slot = self.mem[key]
+            n_el = self._n_el(region, r, q)
+            for j in range(acc.size):
+                if acc[j] or not P.validate_unit(self.enc, slot, j, e):
+                    continue
+                if self.shadow[key][j] != (q, e):
+                    self.violations.append(f"rank {r} epoch {e} accepted {key} unit {j} tagged "
+                                           f"{self.shadow[key][j]}")
+                lo, vals = P.decode_unit(self.enc, slot, j, n_el)
+                rk["staged"][(region, q)][lo:lo + vals.size] = vals
+                acc[j] = True
+                if self.enc == P.SENTINEL and self.sentinel_reset == "on_accept" and self.bug != "no_reset":
+                    off, body = P.reset_unit_bytes(self.enc, j)
+                    slot[off:off + body.size] = body
+                    self.shadow[key][j] = None
+        if not all(acc.all() for (reg, _), acc in rk["acc"].items() if reg == region):
+            return
+        if self.enc == P.SENTINEL and self.sentinel_reset == "after_all" and self.bug != "no_reset":
+            for (reg, q), acc in rk["acc"].items():
+                if reg == region:
+                    key = (region, r, par, q)
+                    for j in range(acc.size):
+                        off, body = P.reset_unit_bytes(self.enc, j)
+                        self.mem[key][off:off + body.size] = body
+                        self.shadow[key][j] = None
+        rk["consumed"][region] = e
+        if region == "rs":
+            lo, hi = self.bounds[r]
+            rows = np.stack([self.inputs[k, q, lo:hi] if q == r else rk["staged"][("rs", q)]
+                             for q in range(self.N)])
+            rk["red"] = reference.allreduce(rows) if hi > lo else np.zeros(0, dtype=np.uint16)
+            rk["phase"] = "ag_push"
+        else:
+            out = np.zeros(self.count, dtype=np.uint16)
+            for q in range(self.N):
+                lo, hi = self.bounds[q]
+                out[lo:hi] = rk["red"] if q == r else rk["staged"][("ag", q)]
+            self.outputs[k, r] = out
+            rk["op"] += 1
+            rk["red"] = None
+            self._begin(r)
+
+    def final_checks(self):
+        v = list(self.violations)
+        if not self.finished():
+            v.append("deadlock: no enabled action while a rank is not done")
+            return v
+        for k in range(self.K):
+            want = reference.allreduce(self.inputs[k])
+            for r in range(self.N):
+                if not np.array_equal(self.outputs[k, r], want):
+                    v.append(f"op {k} rank {r}: output differs from the closed form")
+        if self.enc == P.SENTINEL:
+            for key, buf in self.mem.items():
+                if not np.all(buf == 0xFF):
+                    v.append(f"sentinel slot {key} not reset after the chain")
+        return v
+
+
+def _make_sim(proto, inputs, op, first_epoch, bug, sentinel_reset, vector=8):
+    if proto in SELF_SYNC_TWOSHOT:
+        if op != ALLREDUCE:
+            raise ValueError("twoshot is an all-reduce algorithm")
+        return TwoshotSim(proto, inputs, first_epoch=first_epoch, bug=bug, sentinel_reset=sentinel_reset,
+                          vector=vector)
+    return ChainSim(proto, inputs, op=op, first_epoch=first_epoch, bug=bug, sentinel_reset=sentinel_reset)

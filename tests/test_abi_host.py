@@ -11,7 +11,9 @@ from latency_self_synchronizing_b200 import _lib, api
 from oracle import selector as osel
 
 HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "sfc.h")
-PROTO_NAMES = {1: "ll", 2: "ll128", 3: "sentinel", 4: "barrier_oneshot", 5: "barrier_twoshot"}
+PROTO_NAMES = {1: "ll", 2: "ll128", 3: "sentinel", 4: "barrier_oneshot", 5: "barrier_twoshot",
+               6: "barrier_oneshot_db", 7: "ll_twoshot", 8: "sentinel_twoshot"}
+AR_ONLY = {5, 7, 8}
 
 
 def _declared():
@@ -40,7 +42,7 @@ def test_status_strings():
 def test_algorithmic_bytes_match_oracle(op, n):
     for count in [1, 7, 60, 61, 1024, 8192 * 8, 1 << 20, (1 << 25) + 3]:
         for p, name in PROTO_NAMES.items():
-            if op == "allgather" and p == 5:
+            if op == "allgather" and p in AR_ONLY:
                 assert api.algorithmic_bytes(op, p, count, n) == -1.0
                 continue
             assert api.algorithmic_bytes(op, p, count, n) == pytest.approx(
@@ -51,7 +53,7 @@ def _model_from(entries):
     """ctypes model from {proto: (alpha, beta, table)}; other protocols off."""
     m = api.default_cost_model()
     for op in range(2):
-        for p in range(6):
+        for p in range(9):
             for n in range(9):
                 m.c[op][p][n].alpha_us = -1.0
     for op in range(2):
@@ -86,7 +88,7 @@ def test_cost_estimate_and_selector_match_oracle():
             for n in (2, 5, 8):
                 for b in sizes:
                     for p, name in PROTO_NAMES.items():
-                        if op == "allgather" and name == "barrier_twoshot":
+                        if op == "allgather" and p in AR_ONLY:
                             continue
                         want = osel.estimate(entries[name], name, b, n, op)
                         got = api.cost_estimate(m, op, p, b, n)
@@ -109,4 +111,4 @@ def test_default_model_chooses_a_real_protocol_everywhere():
                 p = api.select_protocol_model(m, op, b, n)
                 assert p != api.Protocol.AUTO
                 if op == "allgather":
-                    assert p != api.Protocol.BARRIER_TWOSHOT
+                    assert int(p) not in AR_ONLY

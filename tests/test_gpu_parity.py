@@ -19,8 +19,9 @@ from _gpu_helpers import Operands, run_chain, slot_bytes
 
 pytestmark = pytest.mark.gpu
 
-AR_PROTOS = ["ll", "ll128", "sentinel", "barrier_oneshot", "barrier_twoshot"]
-AG_PROTOS = ["ll", "ll128", "sentinel", "barrier_oneshot"]
+AR_PROTOS = ["ll", "ll128", "sentinel", "barrier_oneshot", "barrier_twoshot", "barrier_oneshot_db", "ll_twoshot",
+             "sentinel_twoshot"]
+AG_PROTOS = ["ll", "ll128", "sentinel", "barrier_oneshot", "barrier_oneshot_db"]
 RAGGED = [1, 7, 8, 9, 59, 60, 61, 255, 1000, 4099]
 
 
@@ -150,17 +151,19 @@ def test_ll_flags_equal_last_epoch_of_each_parity(comms):
         comm.close()
 
 
-def test_sentinel_slots_reset_after_chain():
+@pytest.mark.parametrize("proto", ["sentinel", "sentinel_twoshot"])
+def test_sentinel_slots_reset_after_chain(proto):
     n, count = 4, 3000
     comm = api.Communicator(n, 1 << 14)
     try:
         x = make_inputs(seed=78, k_ops=7, nranks=n, count=count)
-        _assert_ar(run_chain(comm, "sentinel", x), x)
+        _assert_ar(run_chain(comm, proto, x), x)
+        pars = (0, 1, 2, 3) if proto.endswith("twoshot") else (0, 1)  # twoshot: + all-gather slots
         for r in range(n):
-            for par in (0, 1):
+            for par in pars:
                 for q in range(n):
                     if q != r:
-                        assert np.all(slot_bytes(comm, "sentinel", r, par, q) == 0xFF)
+                        assert np.all(slot_bytes(comm, proto, r, par, q) == 0xFF)
     finally:
         comm.close()
 
@@ -225,7 +228,8 @@ def test_workload_decode_h8192_sentinel_full(tokens):
         comm.close()
 
 
-@pytest.mark.parametrize("proto", ["ll128", "barrier_oneshot", "barrier_twoshot"])
+@pytest.mark.parametrize("proto", ["ll128", "barrier_oneshot", "barrier_twoshot", "ll_twoshot", "sentinel_twoshot",
+                                   "barrier_oneshot_db"])
 @pytest.mark.parametrize("tokens", [1, 4, 16])
 def test_workload_decode_h4096_full(proto, tokens):
     """8 ranks, hidden 4096 x tokens, normal(0,0.5), 64 chained ops."""

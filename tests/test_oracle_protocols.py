@@ -157,3 +157,48 @@ def test_sentinel_reset_on_accept_schedules(n):
         assert not v, v[:3]
     _, v = S.run_chain(P.SENTINEL, x, seed=5, schedule="adversarial", slow_rank=0, sentinel_reset="on_accept")
     assert not v, v[:3]
+
+
+@pytest.mark.parametrize("proto", ["ll_twoshot", "sentinel_twoshot"])
+@pytest.mark.parametrize("n,count,k", [(2, 2, 3), (2, 4, 2)])
+def test_selfsync_twoshot_every_interleaving(proto, n, count, k):
+    """Reduce-scatter + all-gather, both self-synchronizing: every interleaving
+    at two ranks (one-element shards so that every shard carries data)."""
+    x = _x(50 + count, k, n, count)
+    states, v = exhaustive.explore_interleavings(proto, x, max_states=200_000, vector=1)
+    assert not v, v[:3]
+    assert states > 10
+
+
+def test_selfsync_twoshot_catches_missing_reset():
+    x = _x(55, 3, 2, 2)
+    _, v = exhaustive.explore_interleavings("sentinel_twoshot", x, bug="no_reset", vector=1)
+    assert v
+
+
+@pytest.mark.parametrize("proto", ["ll_twoshot", "sentinel_twoshot"])
+@pytest.mark.parametrize("n", [2, 3, 5, 8])
+def test_selfsync_twoshot_schedules(proto, n):
+    x = _x(60 + n, 3, n, 100)  # vector-aligned shards as on the GPU, a ragged tail
+    for seed in range(2):
+        _, v = S.run_chain(proto, x, seed=seed)
+        assert not v, v[:3]
+    _, v = S.run_chain(proto, x, seed=9, schedule="adversarial", slow_rank=n - 1,
+                       sentinel_reset="on_accept")
+    assert not v, v[:3]
+
+
+def test_oneshot_dual_buffer_every_interleaving_and_single_buffer_bug():
+    """SiFAR's dual-buffered oneshot needs no bottom barrier; with one input
+    buffer and no bottom barrier a fast rank overwrites an input a slow rank
+    still pulls."""
+    x = _x(70, 3, 2, 2)
+    states, v = exhaustive.explore_interleavings("barrier_oneshot_db", x)
+    assert not v and states > 10
+    _, v = exhaustive.explore_interleavings("barrier_oneshot_db", x, bug="single_input_buffer")
+    assert v
+    for n in (3, 5, 8):
+        y = _x(71, 4, n, 13)
+        assert not S.run_chain("barrier_oneshot_db", y, seed=1)[1]
+        assert not S.run_chain("barrier_oneshot_db", y, op="allgather", seed=2, schedule="adversarial",
+                               slow_rank=0)[1]
