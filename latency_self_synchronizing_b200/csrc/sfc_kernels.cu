@@ -83,27 +83,84 @@ SFC_DEV uint64_t ll_off(uint64_t v, int half) {
   return ((v >> 5) << 10) + (static_cast<uint64_t>(half) << 9) + ((v & 31) << 4);
 }
 
-// One deferred output vector: the last result of an operation is written
-// after the next operation's pushes, so the per-operation fence does not wait
-// for its store to be acknowledged.
-struct PendingOut {
-  uint16_t* base = nullptr;
-  uint64_t e0 = 0, limit = 0;
-  uint4 v = make_uint4(0, 0, 0, 0);
-  bool valid = false;
-  SFC_DEV void flush() {
-    if (valid) store_n(base, e0, v, 8, limit);
-    valid = false;
+// LL poll + reduce of this thread's vectors, K at a time (all loads of a
+// batch issued before any is examined). K = 1 is what the kernels use:
+// batching several vectors per poll measured no faster on B200, since where a
+// thread owns several vectors the path is bandwidth-bound already. Sources are
+// indexed j = 0..N-2 (q = j or j + 1 around r) so that no register is spent
+// on the own slot.
+template <int N, int OP, int K>
+SFC_DEV bool ll_poll(const KParams& p, int r, int op, uint32_t e, uint64_t gtid, uint64_t gstride,
+                     const uint8_t* my, const uint16_t* in_r, uint16_t* out_r) {
+  const uint64_t count = p.count;
+  const uint64_t nvec = (count + 7) >> 3;
+  const int lane = threadIdx.x & 31;
+  for (uint64_t vb = gtid - lane; vb < nvec; vb += gstride * K) {
+    uint64_t v[K];
+    uint4 own[K];
+    uint32_t need = 0;  // bit i * (N - 1) + j
+#pragma unroll
+    for (int i = 0; i < K; ++i) {
+      v[i] = vb + lane + i * gstride;
+      const bool act = v[i] < nvec;
+      own[i] = act ? load8(in_r, v[i] * 8, count) : make_uint4(0, 0, 0, 0);
+      if (act) need |= ((1u << (N - 1)) - 1u) << (i * (N - 1));
+    }
+    uint64_t a[K][N - 1], b[K][N - 1], c[K][N - 1], d[K][N - 1];
+    WarpWait ww;
+    while (true) {
+      // issue every pending load before looking at any result, so one poll
+      // costs one round trip whatever the number of sources and vectors
+      const uint32_t cur = need;
+#pragma unroll
+      for (int i = 0; i < K; ++i) {
+        const uint64_t o0 = ll_off(v[i], 0), o1 = ll_off(v[i], 1);
+#pragma unroll
+        for (int j = 0; j < N - 1; ++j) {
+          if (cur & (1u << (i * (N - 1) + j))) {
+            const uint8_t* s = my + static_cast<uint64_t>(j) * p.slot_stride;
+            ld_rlx_v2u64(s + o0, a[i][j], b[i][j]);
+            ld_rlx_v2u64(s + o1, c[i][j], d[i][j]);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < K; ++i) {
+#pragma unroll
+        for (int j = 0; j < N - 1; ++j) {
+          const uint32_t bit = 1u << (i * (N - 1) + j);
+          if ((cur & bit) && static_cast<uint32_t>(a[i][j] >> 32) == e && static_cast<uint32_t>(b[i][j] >> 32) == e &&
+              static_cast<uint32_t>(c[i][j] >> 32) == e && static_cast<uint32_t>(d[i][j] >> 32) == e)
+            need &= ~bit;
+        }
+      }
+      if (!__any_sync(kFull, need != 0u)) break;
+      if (ww.tick(p, op, r, need ? (__ffs(need) - 1) % (N - 1) : -1)) return false;
+    }
+#pragma unroll
+    for (int i = 0; i < K; ++i) {
+      if (v[i] >= nvec) continue;
+      uint4 x[N];
+#pragma unroll
+      for (int q = 0; q < N; ++q) {
+        // source q sits at j = q (q < r) or j = q - 1 (q > r)
+        const int jl = q < N - 1 ? q : N - 2, jh = q > 0 ? q - 1 : 0;
+        const uint4 lo = make_uint4(static_cast<uint32_t>(a[i][jl]), static_cast<uint32_t>(b[i][jl]),
+                                    static_cast<uint32_t>(c[i][jl]), static_cast<uint32_t>(d[i][jl]));
+        const uint4 hi = make_uint4(static_cast<uint32_t>(a[i][jh]), static_cast<uint32_t>(b[i][jh]),
+                                    static_cast<uint32_t>(c[i][jh]), static_cast<uint32_t>(d[i][jh]));
+        x[q] = q == r ? own[i] : (q < r ? lo : hi);
+      }
+      if (OP == kAllreduce) {
+        store_n(out_r, v[i] * 8, reduce8<N>(x), 8, count);
+      } else {
+#pragma unroll
+        for (int q = 0; q < N; ++q) store_n(out_r, q * count + v[i] * 8, x[q], 8, q * count + count);
+      }
+    }
   }
-  SFC_DEV void set(uint16_t* b, uint64_t e, uint4 x, uint64_t lim) {
-    flush();
-    base = b;
-    e0 = e;
-    v = x;
-    limit = lim;
-    valid = true;
-  }
-};
+  return true;
+}
 
 // ===================================================================== LL
 // Unit = 8 bytes {2 bf16, epoch}; a 16-byte input vector v becomes units
@@ -111,12 +168,11 @@ struct PendingOut {
 // the two loads equal e.
 template <int N, int OP>
 SFC_DEV bool ll_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid, uint64_t gstride,
-                   const Operands& io, PendingOut& pend) {
+                   const Operands& io) {
   const uint64_t count = p.count;
   const uint64_t nvec = (count + 7) >> 3;
   const int par = e & 1;
   const uint64_t ehi = static_cast<uint64_t>(e) << 32;
-  const int lane = threadIdx.x & 31;
   const uint16_t* in_r = io.in;
   uint16_t* out_r = io.out;
 
@@ -133,63 +189,87 @@ SFC_DEV bool ll_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid, u
       }
     }
   }
-  pend.flush();
   prefetch_next_input(io.in_next, gtid, gstride, nvec);
 
   const uint8_t* my = slot_ptr<N>(p, r, par, r == 0 ? 1 : 0);  // slot j = 0
-  for (uint64_t vb = gtid - lane; vb < nvec; vb += gstride) {
-    const uint64_t v = vb + lane;
-    const bool act = v < nvec;
-    const uint4 own = act ? load8(in_r, v * 8, count) : make_uint4(0, 0, 0, 0);
-    uint32_t need = act ? (((1u << N) - 1u) & ~(1u << r)) : 0u;
-    const uint64_t o0 = ll_off(v, 0), o1 = ll_off(v, 1);
-    // a source's registers keep the units that validated: once accepted it is
-    // not loaded again
-    uint64_t a[N], b[N], c[N], d[N];
+  return ll_poll<N, OP, 1>(p, r, op, e, gtid, gstride, my, in_r, out_r);
+}
+
+// ================================================================ sentinel
+// Sentinel poll + reduce, K vectors at a time, sources indexed j = 0..N-2
+// (as in the LL poll); two bits per (vector, source): its low and high 8-byte
+// unit.
+template <int N, int OP, int K>
+SFC_DEV bool sentinel_poll(const KParams& p, int r, int op, uint64_t gtid, uint64_t gstride, uint8_t* my,
+                           const uint16_t* in_r, uint16_t* out_r) {
+  constexpr uint64_t kFill = ~0ull;
+  const uint64_t count = p.count;
+  const uint64_t nvec = (count + 7) >> 3;
+  const int lane = threadIdx.x & 31;
+  for (uint64_t vb = gtid - lane; vb < nvec; vb += gstride * K) {
+    uint64_t v[K];
+    uint4 own[K];
+    uint32_t need = 0;  // bits 2 * (i * (N - 1) + j) and + 1
+#pragma unroll
+    for (int i = 0; i < K; ++i) {
+      v[i] = vb + lane + i * gstride;
+      const bool act = v[i] < nvec;
+      own[i] = act ? load8(in_r, v[i] * 8, count) : make_uint4(0, 0, 0, 0);
+      if (act) need |= ((1u << (2 * (N - 1))) - 1u) << (2 * i * (N - 1));
+    }
+    uint64_t a[K][N - 1], b[K][N - 1];  // accepted units are never exchanged again
     WarpWait ww;
     while (true) {
-      // issue every pending source's loads before looking at any result, so
-      // one poll costs one round trip whatever the number of sources
+      // every pending exchange is issued before any result is examined
       const uint32_t cur = need;
 #pragma unroll
-      for (int q = 0; q < N; ++q) {
-        if (cur & (1u << q)) {
-          const int j = q < r ? q : q - 1;
-          const uint8_t* s = my + static_cast<uint64_t>(j) * p.slot_stride;
-          ld_rlx_v2u64(s + o0, a[q], b[q]);
-          ld_rlx_v2u64(s + o1, c[q], d[q]);
+      for (int i = 0; i < K; ++i) {
+#pragma unroll
+        for (int j = 0; j < N - 1; ++j) {
+          const int u = 2 * (i * (N - 1) + j);
+          uint8_t* s = my + static_cast<uint64_t>(j) * p.slot_stride + v[i] * 16;
+          if (cur & (1u << u)) a[i][j] = atom_exch_u64(s, kFill);
+          if (cur & (2u << u)) b[i][j] = atom_exch_u64(s + 8, kFill);
         }
       }
 #pragma unroll
-      for (int q = 0; q < N; ++q) {
-        if (cur & (1u << q)) {
-          const bool ok = static_cast<uint32_t>(a[q] >> 32) == e && static_cast<uint32_t>(b[q] >> 32) == e &&
-                          static_cast<uint32_t>(c[q] >> 32) == e && static_cast<uint32_t>(d[q] >> 32) == e;
-          if (ok) need &= ~(1u << q);
+      for (int i = 0; i < K; ++i) {
+#pragma unroll
+        for (int j = 0; j < N - 1; ++j) {
+          const int u = 2 * (i * (N - 1) + j);
+          if ((cur & (1u << u)) && a[i][j] != kFill) need &= ~(1u << u);
+          if ((cur & (2u << u)) && b[i][j] != kFill) need &= ~(2u << u);
         }
       }
       if (!__any_sync(kFull, need != 0u)) break;
-      if (ww.tick(p, op, r, need ? __ffs(need) - 1 : -1)) return false;
+      if (ww.tick(p, op, r, need ? ((__ffs(need) - 1) / 2) % (N - 1) : -1)) return false;
     }
-    if (act) {
+#pragma unroll
+    for (int i = 0; i < K; ++i) {
+      if (v[i] >= nvec) continue;
       uint4 x[N];
 #pragma unroll
-      for (int q = 0; q < N; ++q)
-        x[q] = q == r ? own
-                      : make_uint4(static_cast<uint32_t>(a[q]), static_cast<uint32_t>(b[q]),
-                                   static_cast<uint32_t>(c[q]), static_cast<uint32_t>(d[q]));
+      for (int q = 0; q < N; ++q) {
+        const int jl = q < N - 1 ? q : N - 2, jh = q > 0 ? q - 1 : 0;
+        const uint4 lo = make_uint4(static_cast<uint32_t>(a[i][jl]), static_cast<uint32_t>(a[i][jl] >> 32),
+                                    static_cast<uint32_t>(b[i][jl]), static_cast<uint32_t>(b[i][jl] >> 32));
+        const uint4 hi = make_uint4(static_cast<uint32_t>(a[i][jh]), static_cast<uint32_t>(a[i][jh] >> 32),
+                                    static_cast<uint32_t>(b[i][jh]), static_cast<uint32_t>(b[i][jh] >> 32));
+        x[q] = q == r ? own[i] : (q < r ? lo : hi);
+      }
       if (OP == kAllreduce) {
-        pend.set(out_r, v * 8, reduce8<N>(x), count);
+        store_n(out_r, v[i] * 8, reduce8<N>(x), 8, count);
       } else {
 #pragma unroll
-        for (int q = 0; q < N; ++q) store_n(out_r, q * count + v * 8, x[q], 8, q * count + count);
+        for (int q = 0; q < N; ++q) store_n(out_r, q * count + v[i] * 8, x[q], 8, q * count + count);
       }
     }
   }
   return true;
 }
 
-// ================================================================ sentinel
+
+
 // Raw data into a slot pre-filled with 0xFFFF. The writer moves each 8 bytes
 // as one single-copy-atomic .b64 element, so an 8-byte unit of the slot is
 // either all fill or all data, and data never equals the fill (inputs never
@@ -198,12 +278,10 @@ SFC_DEV bool ll_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid, u
 // the same atomic operation has already written the fill back (the reset).
 template <int N, int OP>
 SFC_DEV bool sentinel_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid, uint64_t gstride,
-                         const Operands& io, PendingOut& pend) {
-  constexpr uint64_t kFill = ~0ull;
+                         const Operands& io) {
   const uint64_t count = p.count;
   const uint64_t nvec = (count + 7) >> 3;
   const int par = e & 1;
-  const int lane = threadIdx.x & 31;
   const uint16_t* in_r = io.in;
   uint16_t* out_r = io.out;
 
@@ -222,57 +300,10 @@ SFC_DEV bool sentinel_op(const KParams& p, int r, int op, uint32_t e, uint64_t g
       }
     }
   }
-  pend.flush();
   prefetch_next_input(io.in_next, gtid, gstride, nvec);
 
   uint8_t* my = slot_ptr<N>(p, r, par, r == 0 ? 1 : 0);
-  for (uint64_t vb = gtid - lane; vb < nvec; vb += gstride) {
-    const uint64_t v = vb + lane;
-    const bool act = v < nvec;
-    const uint4 own = act ? load8(in_r, v * 8, count) : make_uint4(0, 0, 0, 0);
-    // two bits per source: low and high 8-byte unit of the vector
-    uint32_t need = 0;
-    if (act) {
-#pragma unroll
-      for (int q = 0; q < N; ++q)
-        if (q != r) need |= 3u << (2 * q);
-    }
-    uint64_t a[N], b[N];  // keep the accepted units (never exchanged again)
-    WarpWait ww;
-    while (true) {
-      // every pending exchange is issued before any result is examined
-      const uint32_t cur = need;
-#pragma unroll
-      for (int q = 0; q < N; ++q) {
-        const int j = q < r ? q : q - 1;
-        uint8_t* s = my + static_cast<uint64_t>(j) * p.slot_stride + v * 16;
-        if (cur & (1u << (2 * q))) a[q] = atom_exch_u64(s, kFill);
-        if (cur & (2u << (2 * q))) b[q] = atom_exch_u64(s + 8, kFill);
-      }
-#pragma unroll
-      for (int q = 0; q < N; ++q) {
-        if ((cur & (1u << (2 * q))) && a[q] != kFill) need &= ~(1u << (2 * q));
-        if ((cur & (2u << (2 * q))) && b[q] != kFill) need &= ~(2u << (2 * q));
-      }
-      if (!__any_sync(kFull, need != 0u)) break;
-      if (ww.tick(p, op, r, need ? (__ffs(need) - 1) / 2 : -1)) return false;
-    }
-    if (act) {
-      uint4 x[N];
-#pragma unroll
-      for (int q = 0; q < N; ++q)
-        x[q] = q == r ? own
-                      : make_uint4(static_cast<uint32_t>(a[q]), static_cast<uint32_t>(a[q] >> 32),
-                                   static_cast<uint32_t>(b[q]), static_cast<uint32_t>(b[q] >> 32));
-      if (OP == kAllreduce) {
-        pend.set(out_r, v * 8, reduce8<N>(x), count);
-      } else {
-#pragma unroll
-        for (int q = 0; q < N; ++q) store_n(out_r, q * count + v * 8, x[q], 8, q * count + count);
-      }
-    }
-  }
-  return true;
+  return sentinel_poll<N, OP, 1>(p, r, op, gtid, gstride, my, in_r, out_r);
 }
 
 // =================================================================== LL128
@@ -711,7 +742,6 @@ __global__ void __launch_bounds__(kThreads, MinBlocks<N, PROTO>::value) sfc_kern
   if (ld_rlx_s32(&p.status->abort)) return;  // poisoned context: do nothing
   if (p.timings != nullptr && lane == 0)
     atomicMin(reinterpret_cast<unsigned long long*>(&p.timings[0]), static_cast<unsigned long long>(gtimer()));
-  PendingOut pend;
   Operands io{in_ptr<N>(p, 0, r), out_ptr<N>(p, 0, r), nullptr};
   for (int op = 0; op < p.k_ops; ++op) {
     const uint32_t e = p.first_epoch + static_cast<uint32_t>(op);
@@ -720,9 +750,9 @@ __global__ void __launch_bounds__(kThreads, MinBlocks<N, PROTO>::value) sfc_kern
     if (p.skew != nullptr) spin_ns(__ldg(&p.skew[op * N + r]), p.timeout_ns);
     bool ok;
     if (PROTO == kLL)
-      ok = ll_op<N, OP>(p, r, op, e, gtid, gstride, io, pend);
+      ok = ll_op<N, OP>(p, r, op, e, gtid, gstride, io);
     else if (PROTO == kSentinel)
-      ok = sentinel_op<N, OP>(p, r, op, e, gtid, gstride, io, pend);
+      ok = sentinel_op<N, OP>(p, r, op, e, gtid, gstride, io);
     else if (PROTO == kLL128)
       ok = ll128_op<N, OP>(p, r, op, e, gtid, gstride, io);
     else if (PROTO == kOneshot)
@@ -741,7 +771,6 @@ __global__ void __launch_bounds__(kThreads, MinBlocks<N, PROTO>::value) sfc_kern
     if (p.timings != nullptr && lane == 0)
       atomicMax(reinterpret_cast<unsigned long long*>(&p.timings[1 + op]), static_cast<unsigned long long>(gtimer()));
   }
-  pend.flush();
 }
 
 // ============================================================ dispatch table
