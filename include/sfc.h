@@ -66,7 +66,8 @@ typedef enum {
   SFC_ERR_RESOURCES = 5,          /* the ranks' CTAs cannot all be co-resident */
   SFC_ERR_SENTINEL_IN_INPUT = 6,  /* input holds 0xFFFF (debug checks only) */
   SFC_ERR_UNSUPPORTED = 7,        /* protocol / op / dtype combination not provided */
-  SFC_ERR_ABORTED = 8             /* context poisoned by an earlier device error */
+  SFC_ERR_ABORTED = 8,            /* context poisoned by an earlier device error */
+  SFC_ERR_GUARD = 9               /* a scratch guard word was overwritten (sfc_check_guards) */
 } sfc_status;
 
 typedef enum {
@@ -264,6 +265,12 @@ sfc_status sfc_measure_floor(int iters, sfc_floor_result* out);
 
 /* Number of kernel launches this context has issued (all entry points). */
 uint64_t sfc_launch_count(const sfc_ctx* ctx);
+
+/* Every scratch region sits between two 4 KB guards filled with 0xA5 at
+ * sfc_init and never written by any kernel. Synchronizes the context's last
+ * stream and returns SFC_ERR_GUARD if a guard byte changed (a write outside a
+ * region), else SFC_OK. A check for tests and debugging. */
+sfc_status sfc_check_guards(sfc_ctx* ctx);
 
 /* Largest per-rank element count sfc_allreduce_noalloc accepts (8 KB of bf16). */
 #define SFC_NOALLOC_MAX_COUNT 4096

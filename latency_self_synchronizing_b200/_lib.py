@@ -67,6 +67,7 @@ SIGNATURES = [
     ("sfc_set_silent_rank", _S, [_P, C.c_int]),
     ("sfc_measure_floor", _S, [C.c_int, C.POINTER(FloorResult)]),
     ("sfc_launch_count", C.c_uint64, [_P]),
+    ("sfc_check_guards", _S, [_P]),
     ("sfc_allreduce_noalloc", _S, [C.POINTER(_P), C.POINTER(_P), C.c_int, C.c_size_t, _P]),
 ]
 

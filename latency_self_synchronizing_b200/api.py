@@ -28,6 +28,7 @@ class Status(enum.IntEnum):
     SENTINEL_IN_INPUT = 6
     UNSUPPORTED = 7
     ABORTED = 8
+    GUARD = 9
 
 
 class Protocol(enum.IntEnum):
@@ -153,6 +154,10 @@ class Communicator:
         info = C.c_uint32(0)
         rc = self._lib.sfc_get_status(self._ctx, C.byref(info))
         return Status(rc), int(info.value)
+
+    def check_guards(self):
+        """Status of the guard words around the scratch regions."""
+        return Status(self._lib.sfc_check_guards(self._ctx))
 
     @property
     def launch_count(self):

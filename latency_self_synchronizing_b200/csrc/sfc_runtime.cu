@@ -25,6 +25,7 @@ struct sfc_ctx {
   int sm_count = 0;
 
   uint8_t* region[kNumProtocols] = {};  // per self-sync protocol scratch
+  uint8_t* region_raw[kNumProtocols] = {};  // allocation: guard, region, guard
   uint64_t slot_stride[kNumProtocols] = {};
   uint64_t region_bytes[kNumProtocols] = {};
   uint64_t* bar = nullptr;
@@ -54,6 +55,8 @@ namespace {
 constexpr uint32_t kDefaultTimeoutUs = 50000;
 constexpr uint32_t kAllProtocolsMask = ((1u << kNumProtocols) - 1u) & ~1u;
 constexpr int kBarStride = 1024;  // >= any CTAs-per-rank value
+constexpr size_t kGuardBytes = 4096;
+constexpr int kGuardByte = 0xA5;
 
 bool cuda_ok(cudaError_t e) {
   if (e != cudaSuccess) {
@@ -269,6 +272,7 @@ const char* sfc_status_string(sfc_status s) {
     case SFC_ERR_SENTINEL_IN_INPUT: return "input contains the sentinel pattern";
     case SFC_ERR_UNSUPPORTED: return "unsupported protocol, operation or dtype";
     case SFC_ERR_ABORTED: return "context aborted by an earlier device error";
+    case SFC_ERR_GUARD: return "a scratch guard word was overwritten";
   }
   return "unknown status";
 }
@@ -415,7 +419,14 @@ sfc_status sfc_init(sfc_ctx** out, int nranks, size_t max_bytes_per_rank, const 
     c->slot_stride[pr] = sb;
     // twoshot: reduce-scatter slots, then as many all-gather slots
     c->region_bytes[pr] = sb * slots * (pr == kLLTwoshot || pr == kSentinelTwoshot ? 2 : 1);
-    if (!cuda_ok(cudaMalloc(&c->region[pr], c->region_bytes[pr]))) return fail(SFC_ERR_CUDA);
+    // guard words before and after the region catch any write out of it
+    uint8_t* raw = nullptr;
+    if (!cuda_ok(cudaMalloc(&raw, c->region_bytes[pr] + 2 * kGuardBytes))) return fail(SFC_ERR_CUDA);
+    c->region_raw[pr] = raw;
+    c->region[pr] = raw + kGuardBytes;
+    if (!cuda_ok(cudaMemset(raw, kGuardByte, kGuardBytes)) ||
+        !cuda_ok(cudaMemset(raw + kGuardBytes + c->region_bytes[pr], kGuardByte, kGuardBytes)))
+      return fail(SFC_ERR_CUDA);
   }
   c->bar_stride = kBarStride;
   if (!cuda_ok(cudaMalloc(&c->bar, sizeof(uint64_t) * nranks * kBarStride))) return fail(SFC_ERR_CUDA);
@@ -436,9 +447,10 @@ sfc_status sfc_init(sfc_ctx** out, int nranks, size_t max_bytes_per_rank, const 
 sfc_status sfc_destroy(sfc_ctx* c) {
   if (c == nullptr) return SFC_ERR_INVALID;
   (void)cudaDeviceSynchronize();
-  for (auto& r : c->region) {
-    if (r) cudaFree(r);
-    r = nullptr;
+  for (int pr = 0; pr < kNumProtocols; ++pr) {
+    if (c->region_raw[pr]) cudaFree(c->region_raw[pr]);
+    c->region_raw[pr] = nullptr;
+    c->region[pr] = nullptr;
   }
   if (c->bar) cudaFree(c->bar);
   if (c->red) cudaFree(c->red);
@@ -589,5 +601,20 @@ sfc_status sfc_set_silent_rank(sfc_ctx* c, int silent_rank) {
 }
 
 uint64_t sfc_launch_count(const sfc_ctx* c) { return c ? c->launches : 0; }
+
+sfc_status sfc_check_guards(sfc_ctx* c) {
+  if (c == nullptr) return SFC_ERR_INVALID;
+  if (!cuda_ok(cudaStreamSynchronize(c->last_stream))) return SFC_ERR_CUDA;
+  std::vector<uint8_t> h(kGuardBytes);
+  for (int pr = 0; pr < kNumProtocols; ++pr) {
+    if (c->region_raw[pr] == nullptr) continue;
+    for (uint8_t* g : {c->region_raw[pr], c->region[pr] + c->region_bytes[pr]}) {
+      if (!cuda_ok(cudaMemcpy(h.data(), g, kGuardBytes, cudaMemcpyDeviceToHost))) return SFC_ERR_CUDA;
+      for (uint8_t b : h)
+        if (b != kGuardByte) return SFC_ERR_GUARD;
+    }
+  }
+  return SFC_OK;
+}
 
 }  // extern "C"

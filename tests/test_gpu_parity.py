@@ -294,3 +294,14 @@ def test_timings_are_monotone(comms):
     h = t.cpu().numpy().astype(np.uint64)
     assert np.all(np.diff(h[1:].astype(np.int64)) >= 0)
     assert h[1] >= h[0]
+
+
+@pytest.mark.parametrize("proto", AR_PROTOS)
+def test_guard_words_intact_after_large_chain(proto):
+    comm = api.Communicator(8, 1 << 18, protocols=[proto])
+    try:
+        x = make_inputs(seed=91, k_ops=3, nranks=8, count=(1 << 17) - 3)
+        _assert_ar(run_chain(comm, proto, x), x)
+        assert comm.check_guards() == api.Status.OK
+    finally:
+        comm.close()

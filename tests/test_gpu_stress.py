@@ -1,0 +1,59 @@
+"""Long-run robustness on the GPU: a million chained operations per
+self-synchronizing protocol under random per-(operation, rank) start skew,
+every output checked against the oracle, guard words intact afterwards.
+
+The readiness logic is the part that could tear or race (a unit accepted
+before all of it landed, a slot reused too early); the skew makes ranks
+arrive in changing orders. Outputs are compared on the device with torch,
+against expected values the CPU oracle computed for each distinct input set.
+"""
+import numpy as np
+import pytest
+import torch
+
+from latency_self_synchronizing_b200 import api
+from latency_self_synchronizing_b200.inputs import make_inputs
+from oracle import reference
+
+from _gpu_helpers import Operands
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(proto, n, count, total_ops, skew_mean_ns, seed):
+    sets = 64  # distinct input sets; operation i uses set i % 64 and output slot i % 64
+    x = make_inputs(seed=seed, k_ops=sets, nranks=n, count=count)
+    want = np.stack([reference.allreduce(x[s]) for s in range(sets)])  # [sets, count]
+    comm = api.Communicator(n, 2 * count)
+    try:
+        ins = Operands(sets, n, count, fill=x)
+        outs = Operands(sets, n, count)
+        view = outs.buf.view(sets, n, outs.stride)[:, :, :count]
+        want_dev = torch.from_numpy(want.view(np.int16)).cuda()[:, None, :].expand(sets, n, count)
+        rng = np.random.default_rng(seed)
+        skews = [torch.from_numpy(rng.exponential(skew_mean_ns, size=sets * n).astype(np.int32)).cuda()
+                 for _ in range(16)]
+        bad = torch.zeros((), dtype=torch.int64, device="cuda")
+        launches = total_ops // sets
+        for i in range(launches):
+            comm.allreduce_chain(ins.table, outs.table, count, sets, protocol=proto, skew_ns=skews[i % 16])
+            bad += (view != want_dev).sum()
+            view.zero_()
+        torch.cuda.synchronize()
+        st, info = comm.status()
+        assert st == api.Status.OK, (st, hex(info))
+        assert int(bad) == 0, f"{int(bad)} wrong elements over {launches * sets} operations"
+        assert comm.check_guards() == api.Status.OK
+        assert comm.next_epoch == 1 + launches * sets
+    finally:
+        comm.close()
+
+
+@pytest.mark.parametrize("proto", ["ll", "ll128", "sentinel", "ll_twoshot", "sentinel_twoshot"])
+def test_million_ops_under_skew(proto):
+    _run(proto, n=4, count=1000, total_ops=1_000_000, skew_mean_ns=300.0, seed=7)
+
+
+@pytest.mark.parametrize("proto", ["ll", "sentinel", "barrier_oneshot", "barrier_oneshot_db", "barrier_twoshot"])
+def test_many_ops_eight_ranks(proto):
+    _run(proto, n=8, count=4099, total_ops=1 << 17, skew_mean_ns=1000.0, seed=8)
