@@ -266,6 +266,41 @@ sfc_status sfc_measure_floor(int iters, sfc_floor_result* out);
 /* Number of kernel launches this context has issued (all entry points). */
 uint64_t sfc_launch_count(const sfc_ctx* ctx);
 
+/* Device-side LL view of a context, for user kernels that push and poll LL
+ * units themselves through the device API in sfc_ll_device.cuh ("Why
+ * Microseconds Matter in AI Infrastructure", section "Communication is
+ * becoming part of GPU execution": LL send / receive / reduce called from
+ * inside kernels). Plain data; valid while the context lives. */
+typedef struct {
+  unsigned char* scratch;   /* LL region; slot (recv, parity, j) at
+                               ((recv * 2 + parity) * (nranks - 1) + j) * slot_stride,
+                               j = src < recv ? src : src - 1 */
+  uint64_t slot_stride;     /* bytes */
+  int nranks;
+  int* status;              /* {first error, detail, abort word, unused} */
+  uint64_t timeout_ns;      /* bound on each device-side wait */
+} sfc_ll_view;
+
+/* Fill *view for the context's LL scratch (SFC_ERR_UNSUPPORTED if LL is not
+ * provisioned). */
+sfc_status sfc_get_ll_view(sfc_ctx* ctx, sfc_ll_view* view);
+
+/* Reserve k consecutive epochs for a user kernel that uses the LL view:
+ * *first receives the first; the context's next epoch advances by k. */
+sfc_status sfc_reserve_epochs(sfc_ctx* ctx, uint32_t k, uint32_t* first);
+
+/* Row-parallel linear layer fused with its all-reduce, for one decode token:
+ * every rank r holds W[r] (bf16 [hidden][kdim], row-major: its slice of the
+ * input dimension) and x[r] (bf16 [kdim]); the kernel computes the partial
+ * p_r = bf16_RNE(W[r] x[r]) (fp32 accumulation) and, from the registers that
+ * hold it, pushes it as LL units to every peer; each rank then polls,
+ * reduces p_0..p_{N-1} in rank order in fp32 and writes y[r] (bf16
+ * [hidden], identical on every rank). One launch, no intermediate buffer.
+ * hidden % 8 == 0, hidden <= max count of the context; kdim % 8 == 0,
+ * kdim <= 49152; all pointers 16-byte aligned; consumes one epoch. */
+sfc_status sfc_linear_allreduce(sfc_ctx* ctx, const void* const* W, const void* const* x, void* const* y,
+                                size_t hidden, size_t kdim, uint32_t epoch, void* stream);
+
 /* Every scratch region sits between two 4 KB guards filled with 0xA5 at
  * sfc_init and never written by any kernel. Synchronizes the context's last
  * stream and returns SFC_ERR_GUARD if a guard byte changed (a write outside a

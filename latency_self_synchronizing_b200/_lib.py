@@ -34,6 +34,11 @@ class CostModel(C.Structure):
     _fields_ = [("c", CostEntry * (SFC_MAX_RANKS + 1) * SFC_NUM_PROTOCOLS * 2)]
 
 
+class LLView(C.Structure):
+    _fields_ = [("scratch", C.c_void_p), ("slot_stride", C.c_uint64), ("nranks", C.c_int),
+                ("status", C.c_void_p), ("timeout_ns", C.c_uint64)]
+
+
 class FloorResult(C.Structure):
     _fields_ = [("flag_rtt_ns_p50", C.c_double), ("flag_rtt_ns_p99", C.c_double),
                 ("flag_rtt_ns_min_pair", C.c_double), ("flag_rtt_ns_max_pair", C.c_double), ("pairs", C.c_int),
@@ -68,6 +73,10 @@ SIGNATURES = [
     ("sfc_measure_floor", _S, [C.c_int, C.POINTER(FloorResult)]),
     ("sfc_launch_count", C.c_uint64, [_P]),
     ("sfc_check_guards", _S, [_P]),
+    ("sfc_get_ll_view", _S, [_P, C.POINTER(LLView)]),
+    ("sfc_reserve_epochs", _S, [_P, C.c_uint32, C.POINTER(C.c_uint32)]),
+    ("sfc_linear_allreduce", _S, [_P, C.POINTER(_P), C.POINTER(_P), C.POINTER(_P), C.c_size_t, C.c_size_t,
+                                  C.c_uint32, _P]),
     ("sfc_allreduce_noalloc", _S, [C.POINTER(_P), C.POINTER(_P), C.c_int, C.c_size_t, _P]),
 ]
 

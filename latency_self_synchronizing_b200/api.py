@@ -236,6 +236,34 @@ class Communicator:
                                                   int(as_protocol(protocol)), e, tim_p, _stream_handle(stream)),
                "sfc_allreduce_chain_host")
 
+    def linear_allreduce(self, weights, xs, ys, epoch=None, stream=None):
+        """Fused row-parallel linear + all-reduce for one token:
+        ys[r] = sum over ranks of bf16(weights[q] @ xs[q]) (rank order, one
+        rounding), weights[r] [hidden, kdim], xs[r] [kdim], ys[r] [hidden]."""
+        n = self.nranks
+        if not (len(weights) == len(xs) == len(ys) == n):
+            raise ValueError(f"need {n} weights, inputs and outputs")
+        hidden, kdim = weights[0].shape
+        for w, x_, y_ in zip(weights, xs, ys):
+            if tuple(w.shape) != (hidden, kdim) or x_.numel() != kdim or y_.numel() != hidden:
+                raise ValueError("shape mismatch")
+        W = (C.c_void_p * n)(*[_dev_ptr(w, "weight") for w in weights])
+        X = (C.c_void_p * n)(*[_dev_ptr(t, "input") for t in xs])
+        Y = (C.c_void_p * n)(*[_dev_ptr(t, "output") for t in ys])
+        e = self.next_epoch if epoch is None else int(epoch)
+        _check(self._lib.sfc_linear_allreduce(self._ctx, W, X, Y, int(hidden), int(kdim), e, _stream_handle(stream)),
+               "sfc_linear_allreduce")
+
+    def ll_view(self):
+        v = _lib.LLView()
+        _check(self._lib.sfc_get_ll_view(self._ctx, C.byref(v)), "sfc_get_ll_view")
+        return v
+
+    def reserve_epochs(self, k):
+        first = C.c_uint32(0)
+        _check(self._lib.sfc_reserve_epochs(self._ctx, int(k), C.byref(first)), "sfc_reserve_epochs")
+        return int(first.value)
+
     # ------------------------------------------------------------- helpers
     def select_protocol(self, op, bytes_per_rank, nranks=None):
         n = self.nranks if nranks is None else int(nranks)

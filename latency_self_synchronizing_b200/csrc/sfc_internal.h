@@ -1,8 +1,12 @@
 // Internal definitions shared by the host runtime and the kernels of libsfc.
 #pragma once
 
+#include <cuda_runtime.h>
+
 #include <cstddef>
 #include <cstdint>
+
+#include "sfc.h"
 
 namespace sfc {
 
@@ -86,6 +90,20 @@ struct KParams {
   int debug;
   int silent_rank;      // -1 = none
 };
+
+// Fused row-parallel linear + LL all-reduce (one decode token).
+struct LinearParams {
+  const uint16_t* W[kMaxRanks];  // [hidden][kdim] row-major, per rank
+  const uint16_t* x[kMaxRanks];  // [kdim], per rank
+  uint16_t* y[kMaxRanks];        // [hidden], per rank
+  uint64_t hidden;
+  uint64_t kdim;
+  int G;                         // CTAs per rank
+  uint32_t epoch;
+  sfc_ll_view view;
+};
+constexpr int kLinearThreads = 256;
+const void* linear_kernel_for(int nranks);
 
 // Kernel entry for (nranks, protocol, op); null if not provided.
 const void* kernel_for(int nranks, int protocol, int op);

@@ -37,6 +37,7 @@
 #include <cuda_runtime.h>
 
 #include "sfc_device.cuh"
+#include "sfc_ll_device.cuh"
 
 namespace sfc {
 
@@ -79,9 +80,8 @@ struct Operands {
   const uint16_t* in_next;  // null on the last operation
 };
 
-SFC_DEV uint64_t ll_off(uint64_t v, int half) {
-  return ((v >> 5) << 10) + (static_cast<uint64_t>(half) << 9) + ((v & 31) << 4);
-}
+// LL layout shared with the public device API (one definition).
+SFC_DEV uint64_t ll_off(uint64_t v, int half) { return sfc_device::ll_offset(v, half); }
 
 // LL poll + reduce of this thread's vectors, K at a time (all loads of a
 // batch issued before any is examined). K = 1 is what the kernels use:

@@ -602,6 +602,81 @@ sfc_status sfc_set_silent_rank(sfc_ctx* c, int silent_rank) {
 
 uint64_t sfc_launch_count(const sfc_ctx* c) { return c ? c->launches : 0; }
 
+sfc_status sfc_get_ll_view(sfc_ctx* c, sfc_ll_view* view) {
+  if (c == nullptr || view == nullptr) return SFC_ERR_INVALID;
+  if (c->region[kLL] == nullptr) return SFC_ERR_UNSUPPORTED;
+  view->scratch = c->region[kLL];
+  view->slot_stride = c->slot_stride[kLL];
+  view->nranks = c->nranks;
+  view->status = reinterpret_cast<int*>(c->dstatus);
+  view->timeout_ns = static_cast<uint64_t>(c->cfg.timeout_us ? c->cfg.timeout_us : kDefaultTimeoutUs) * 1000ull;
+  return SFC_OK;
+}
+
+sfc_status sfc_reserve_epochs(sfc_ctx* c, uint32_t k, uint32_t* first) {
+  if (c == nullptr || first == nullptr || k == 0) return SFC_ERR_INVALID;
+  if (c->poisoned) return SFC_ERR_ABORTED;
+  if (static_cast<uint64_t>(c->next_epoch) + k - 1 > 0xFFFFFFFFull) return SFC_ERR_EPOCH;
+  *first = c->next_epoch;
+  c->next_epoch += k;
+  return SFC_OK;
+}
+
+sfc_status sfc_linear_allreduce(sfc_ctx* c, const void* const* W, const void* const* x, void* const* y,
+                                size_t hidden, size_t kdim, uint32_t epoch, void* stream) {
+  if (c == nullptr || W == nullptr || x == nullptr || y == nullptr) return SFC_ERR_INVALID;
+  if (hidden == 0 || hidden % 8 || hidden > c->max_count || kdim == 0 || kdim % 8 || kdim > 49152)
+    return SFC_ERR_INVALID;
+  if (c->region[kLL] == nullptr) return SFC_ERR_UNSUPPORTED;
+  if (c->poisoned) return SFC_ERR_ABORTED;
+  if (epoch != c->next_epoch) return SFC_ERR_EPOCH;
+  const int N = c->nranks;
+  sfc::LinearParams p{};
+  for (int r = 0; r < N; ++r) {
+    if (!W[r] || !x[r] || !y[r] || !aligned16(W[r]) || !aligned16(x[r]) || !aligned16(y[r])) return SFC_ERR_INVALID;
+    p.W[r] = static_cast<const uint16_t*>(W[r]);
+    p.x[r] = static_cast<const uint16_t*>(x[r]);
+    p.y[r] = static_cast<uint16_t*>(y[r]);
+  }
+  for (int a = 0; a < N; ++a)
+    for (int b = 0; b < N; ++b)
+      if (overlap(y[a], hidden * 2, x[b], kdim * 2) || overlap(y[a], hidden * 2, W[b], hidden * kdim * 2) ||
+          (a < b && overlap(y[a], hidden * 2, y[b], hidden * 2)))
+        return SFC_ERR_INVALID;
+  const void* fn = linear_kernel_for(N);
+  const int smem = static_cast<int>(kdim * 2);
+  if (smem > 48 * 1024 &&
+      !cuda_ok(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
+    return SFC_ERR_CUDA;
+  int occ = 0;
+  if (!cuda_ok(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kLinearThreads, smem)) || occ < 1)
+    return SFC_ERR_RESOURCES;
+  // every SM streams weights: as many CTAs per rank as can be co-resident,
+  // but no more warps than output vectors
+  const int gmax = occ * c->sm_count / N;
+  const uint64_t warps_needed = (hidden / 8);
+  const int G = static_cast<int>(std::min<uint64_t>(gmax, (warps_needed + 7) / 8));
+  if (G < 1) return SFC_ERR_RESOURCES;
+  p.hidden = hidden;
+  p.kdim = kdim;
+  p.G = G;
+  p.epoch = epoch;
+  sfc_status s = sfc_get_ll_view(c, &p.view);
+  if (s != SFC_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* args[] = {&p};
+  cudaError_t e = cudaLaunchCooperativeKernel(fn, dim3(N * G), dim3(kLinearThreads), args, smem, st);
+  if (e == cudaErrorCooperativeLaunchTooLarge) {
+    (void)cudaGetLastError();
+    return SFC_ERR_RESOURCES;
+  }
+  if (!cuda_ok(e)) return SFC_ERR_CUDA;
+  c->launches++;
+  c->last_stream = st;
+  c->next_epoch = epoch + 1;
+  return SFC_OK;
+}
+
 sfc_status sfc_check_guards(sfc_ctx* c) {
   if (c == nullptr) return SFC_ERR_INVALID;
   if (!cuda_ok(cudaStreamSynchronize(c->last_stream))) return SFC_ERR_CUDA;

@@ -1,0 +1,83 @@
+"""The fused row-parallel linear + all-reduce (one decode token) against an
+fp64 reference of the same product and sum.
+
+The partial products are fp32 accumulations whose order is the kernel's, so
+they are not bit-exact to any plain definition; the all-reduce of them is.
+Bound used (per output element): each rank's partial p_r is within
+2^-8 |d_r| + kdim 2^-24 a_r of the exact dot product d_r (one bf16 rounding,
+kdim fp32 roundings of partial sums bounded by a_r = sum_i |W_ri x_ri|), and
+the rank-order all-reduce of the partials is within 2^-7 N sum_r |p_r| of
+their exact sum. Every rank's output must be bit-identical.
+"""
+import numpy as np
+import pytest
+import torch
+
+from latency_self_synchronizing_b200 import api
+from latency_self_synchronizing_b200.inputs import make_inputs
+from oracle.bf16 import bf16_bits_to_f32
+
+pytestmark = pytest.mark.gpu
+
+
+def _bf16_dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def _case(n, hidden, kdim, seed):
+    w = make_inputs(seed=seed, k_ops=1, nranks=n, count=hidden * kdim, dist="normal", params=(0.05,))[0]
+    x = make_inputs(seed=seed + 1, k_ops=1, nranks=n, count=kdim, dist="normal", params=(1.0,))[0]
+    return w.reshape(n, hidden, kdim), x
+
+
+@pytest.mark.parametrize("n,hidden,kdim", [(2, 8, 8), (2, 1000, 512), (4, 8192, 7168), (8, 4096, 1024),
+                                           (3, 2056, 136), (8, 24, 8)])
+def test_linear_allreduce_within_bound(n, hidden, kdim):
+    w, x = _case(n, hidden, kdim, seed=hidden + kdim + n)
+    comm = api.Communicator(n, hidden * 2, protocols=["ll"])
+    try:
+        W = [_bf16_dev(w[r]) for r in range(n)]
+        X = [_bf16_dev(x[r]) for r in range(n)]
+        Y = [torch.empty(hidden, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+        for _ in range(2):  # two epochs in a row
+            comm.linear_allreduce(W, X, Y)
+            torch.cuda.synchronize()
+            assert comm.status()[0] == api.Status.OK
+            ys = [Y[r].cpu().view(torch.int16).numpy().view(np.uint16) for r in range(n)]
+            for r in range(1, n):
+                np.testing.assert_array_equal(ys[r], ys[0])
+            wf = bf16_bits_to_f32(w).astype(np.float64)
+            xf = bf16_bits_to_f32(x).astype(np.float64)
+            d = np.einsum("rhk,rk->rh", wf, xf)               # exact enough in fp64
+            a = np.einsum("rhk,rk->rh", np.abs(wf), np.abs(xf))
+            eps = 2.0 ** -8 * np.abs(d) + kdim * 2.0 ** -24 * a
+            bound = eps.sum(0) + 2.0 ** -7 * n * (np.abs(d) + eps).sum(0)
+            got = bf16_bits_to_f32(ys[0]).astype(np.float64)
+            assert np.all(np.abs(got - d.sum(0)) <= bound)
+    finally:
+        comm.close()
+
+
+def test_linear_allreduce_shares_the_epoch_sequence():
+    n, hidden, kdim = 4, 64, 64
+    w, x = _case(n, hidden, kdim, seed=5)
+    comm = api.Communicator(n, 4096)
+    try:
+        W = [_bf16_dev(w[r]) for r in range(n)]
+        X = [_bf16_dev(x[r]) for r in range(n)]
+        Y = [torch.empty(hidden, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+        e = comm.next_epoch
+        comm.linear_allreduce(W, X, Y)
+        assert comm.next_epoch == e + 1
+        first = comm.reserve_epochs(3)
+        assert first == e + 1 and comm.next_epoch == e + 4
+        with pytest.raises(api.SfcError) as ei:
+            comm.linear_allreduce(W, X, Y, epoch=e)
+        assert ei.value.status == api.Status.EPOCH
+        comm.linear_allreduce(W, X, Y)  # LL flags of the reserved epochs never appeared: still fine
+        torch.cuda.synchronize()
+        assert comm.status()[0] == api.Status.OK
+        view = comm.ll_view()
+        assert view.nranks == n and view.slot_stride > 0
+    finally:
+        comm.close()
