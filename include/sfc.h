@@ -86,10 +86,18 @@ typedef enum {
   /* all-reduce only: reduce-scatter then all-gather, each phase a
    * self-synchronizing push with LL or sentinel readiness; no barrier */
   SFC_PROTO_LL_TWOSHOT = 7,
-  SFC_PROTO_SENTINEL_TWOSHOT = 8
+  SFC_PROTO_SENTINEL_TWOSHOT = 8,
+  /* LL128 lines written and read with one warp-wide 16-byte-per-lane access
+   * and no fences, relying on a 128-byte line being observed whole (not
+   * promised by the PTX memory model; checked on B200 by a skewed
+   * million-operation stress test). Opt-in: the built-in selector model
+   * holds its measured latencies but marks it unavailable (alpha_us = -1);
+   * a caller who accepts the assumption sets alpha_us = 0 in the entries it
+   * wants and installs the model with sfc_set_cost_model. */
+  SFC_PROTO_LL128_FAST = 9
 } sfc_protocol;
 
-#define SFC_NUM_PROTOCOLS 9
+#define SFC_NUM_PROTOCOLS 10
 #define SFC_MAX_RANKS 8
 
 typedef enum { SFC_BF16 = 0 } sfc_dtype;
@@ -203,8 +211,9 @@ sfc_status sfc_allreduce_chain_host(sfc_ctx* ctx, int k_ops, const void* in_host
  * Decoding", abstract; the empirical choice in "Why Microseconds Matter in AI
  * Infrastructure", section "What I learned from it"). argmin over protocols
  * of the model's latency estimate (sfc_cost_estimate); ties go to fewer
- * algorithmic bytes, then to the order SENTINEL, LL128, LL, SENTINEL_TWOSHOT,
- * LL_TWOSHOT, BARRIER_ONESHOT_DB, BARRIER_ONESHOT, BARRIER_TWOSHOT. Host only. */
+ * algorithmic bytes, then to the order SENTINEL, LL128, LL128_FAST, LL,
+ * SENTINEL_TWOSHOT, LL_TWOSHOT, BARRIER_ONESHOT_DB, BARRIER_ONESHOT,
+ * BARRIER_TWOSHOT. Host only. */
 sfc_protocol sfc_select_protocol(const sfc_ctx* ctx, sfc_op op, size_t bytes_per_rank, int nranks);
 
 /* The same choice from an explicit model; needs no context and no GPU. */

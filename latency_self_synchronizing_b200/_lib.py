@@ -12,7 +12,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 # SFC_LIB selects another build of the same library (e.g. a debug build).
 LIB_PATH = os.environ.get("SFC_LIB") or os.path.join(_HERE, "libsfc.so")
 
-SFC_NUM_PROTOCOLS = 9
+SFC_NUM_PROTOCOLS = 10
 SFC_MAX_RANKS = 8
 
 

@@ -41,6 +41,7 @@ class Protocol(enum.IntEnum):
     BARRIER_ONESHOT_DB = 6
     LL_TWOSHOT = 7
     SENTINEL_TWOSHOT = 8
+    LL128_FAST = 9
 
 
 class Op(enum.IntEnum):
@@ -52,7 +53,8 @@ _NAMES = {"auto": Protocol.AUTO, "ll": Protocol.LL, "ll128": Protocol.LL128, "se
           "barrier_oneshot": Protocol.BARRIER_ONESHOT, "oneshot": Protocol.BARRIER_ONESHOT,
           "barrier_twoshot": Protocol.BARRIER_TWOSHOT, "twoshot": Protocol.BARRIER_TWOSHOT,
           "barrier_oneshot_db": Protocol.BARRIER_ONESHOT_DB, "oneshot_db": Protocol.BARRIER_ONESHOT_DB,
-          "ll_twoshot": Protocol.LL_TWOSHOT, "sentinel_twoshot": Protocol.SENTINEL_TWOSHOT}
+          "ll_twoshot": Protocol.LL_TWOSHOT, "sentinel_twoshot": Protocol.SENTINEL_TWOSHOT,
+          "ll128_fast": Protocol.LL128_FAST}
 
 
 def as_protocol(p):

@@ -24,7 +24,8 @@ enum : int {
   kOneshotDB = 6,
   kLLTwoshot = 7,
   kSentinelTwoshot = 8,
-  kNumProtocols = 9
+  kLL128Fast = 9,
+  kNumProtocols = 10
 };
 // operations (match sfc_op)
 enum : int { kAllreduce = 0, kAllgather = 1 };

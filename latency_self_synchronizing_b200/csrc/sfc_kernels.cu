@@ -622,6 +622,108 @@ SFC_DEV bool selfsync_twoshot_op(const KParams& p, int r, int op, uint32_t e, ui
   return true;
 }
 
+// ============================================================ LL128, one load
+// The same line layout, moved the way the "LL128 atomic design" of "Why
+// Microseconds Matter in AI Infrastructure" (section "Latency can matter more
+// than bandwidth") is built: the 8 lanes of a line store their 16 bytes (lane
+// 7: 8 data bytes + the flag) in one warp-wide store instruction, and a reader
+// takes the whole line with one warp-wide load, accepting the data read in
+// the same instruction as a matching flag. No fence on either side. The PTX
+// memory model does not promise that a 128-byte line written by one warp
+// instruction is observed whole; this protocol relies on B200 behaving so
+// (writes and reads of one line are single L2 requests), which the skewed
+// million-operation stress test checks bit for bit. Opt-in only: the
+// selector never picks it by default.
+template <int N, int OP>
+SFC_DEV bool ll128_fast_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid, uint64_t gstride,
+                           const Operands& io) {
+  const uint64_t count = p.count;
+  const uint64_t nlines = (count + kLL128Elems - 1) / kLL128Elems;
+  const uint64_t ngroups = (nlines + kLL128LinesPerWarp - 1) / kLL128LinesPerWarp;
+  const int par = e & 1;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane & 7;
+  const int lead = lane | 7;  // the flag lane of this lane's line
+  const uint64_t lsel = static_cast<uint64_t>(lane >> 3);
+  const uint64_t wg = gtid >> 5, wstride = gstride >> 5;
+  const uint16_t* in_r = io.in;
+  uint16_t* out_r = io.out;
+
+  if (r != p.silent_rank) {
+    for (uint64_t g = wg; g < ngroups; g += wstride) {
+      const uint64_t L = g * kLL128LinesPerWarp + lsel;
+      if (L < nlines) {
+        const uint64_t e0 = L * kLL128Elems + sub * 8;
+        const uint2 lo = load4(in_r, e0, count);
+        const uint2 hi = sub < 7 ? load4(in_r, e0 + 4, count) : make_uint2(static_cast<uint32_t>(e), 0u);
+        const uint64_t a = (static_cast<uint64_t>(lo.y) << 32) | lo.x;
+        const uint64_t b = (static_cast<uint64_t>(hi.y) << 32) | hi.x;
+#pragma unroll
+        for (int q = 0; q < N; ++q) {
+          if (q == r) continue;
+          st_rlx_v2u64(slot_ptr<N>(p, q, par, r) + L * kLL128Line + sub * 16, a, b);
+        }
+      }
+    }
+  }
+  if (io.in_next != nullptr) {
+    int n = 0;
+    for (uint64_t g = wg; g < ngroups && n < 8; g += wstride, ++n) {
+      const uint64_t L = g * kLL128LinesPerWarp + lsel;
+      const uint64_t e0 = L * kLL128Elems + sub * 8;
+      if (L < nlines && e0 < count) prefetch_l2(io.in_next + e0);
+    }
+  }
+
+  const uint8_t* my = slot_ptr<N>(p, r, par, r == 0 ? 1 : 0);
+  for (uint64_t g = wg; g < ngroups; g += wstride) {
+    const uint64_t L = g * kLL128LinesPerWarp + lsel;
+    const bool has = L < nlines;
+    uint32_t need = has ? ((1u << (N - 1)) - 1u) : 0u;  // bit j: source j pending for this line
+    uint64_t a[N - 1], b[N - 1];
+    WarpWait ww;
+    while (true) {
+      const uint32_t cur = need;
+#pragma unroll
+      for (int j = 0; j < N - 1; ++j)
+        if (cur & (1u << j))
+          ld_rlx_v2u64(my + static_cast<uint64_t>(j) * p.slot_stride + L * kLL128Line + sub * 16, a[j], b[j]);
+      // the flag lane decides for its line; the other 7 lanes take its verdict
+      uint32_t okbits = 0;
+#pragma unroll
+      for (int j = 0; j < N - 1; ++j)
+        if ((cur & (1u << j)) && b[j] == static_cast<uint64_t>(e)) okbits |= 1u << j;
+      okbits = __shfl_sync(kFull, okbits, lead);
+      need &= ~okbits;
+      if (!__any_sync(kFull, need != 0u)) break;
+      if (ww.tick(p, op, r, -1)) return false;
+    }
+    if (!has) continue;
+    const uint64_t e0 = L * kLL128Elems + sub * 8;
+    const int n = sub < 7 ? 8 : 4;
+    const uint2 olo = load4(in_r, e0, count);
+    const uint2 ohi = sub < 7 ? load4(in_r, e0 + 4, count) : make_uint2(0u, 0u);
+    uint4 x[N];
+#pragma unroll
+    for (int q = 0; q < N; ++q) {
+      const int jl = q < N - 1 ? q : N - 2, jh = q > 0 ? q - 1 : 0;
+      const bool below = q < r;
+      const uint64_t va = below ? a[jl] : a[jh];
+      const uint64_t vb = below ? b[jl] : b[jh];
+      x[q] = make_uint4(static_cast<uint32_t>(va), static_cast<uint32_t>(va >> 32),
+                        sub < 7 ? static_cast<uint32_t>(vb) : 0u, sub < 7 ? static_cast<uint32_t>(vb >> 32) : 0u);
+      if (q == r) x[q] = make_uint4(olo.x, olo.y, ohi.x, ohi.y);
+    }
+    if (OP == kAllreduce) {
+      store_n(out_r, e0, reduce8<N>(x), n, count);
+    } else {
+#pragma unroll
+      for (int q = 0; q < N; ++q) store_n(out_r, q * count + e0, x[q], n, q * count + count);
+    }
+  }
+  return true;
+}
+
 // ============================================================ barriers
 // Per-CTA-index barrier: CTA k of rank r publishes (epoch << 2) | phase with
 // a release store and waits until CTA k of every rank has published at least
@@ -755,6 +857,8 @@ __global__ void __launch_bounds__(kThreads, MinBlocks<N, PROTO>::value) sfc_kern
       ok = sentinel_op<N, OP>(p, r, op, e, gtid, gstride, io);
     else if (PROTO == kLL128)
       ok = ll128_op<N, OP>(p, r, op, e, gtid, gstride, io);
+    else if (PROTO == kLL128Fast)
+      ok = ll128_fast_op<N, OP>(p, r, op, e, gtid, gstride, io);
     else if (PROTO == kOneshot)
       ok = oneshot_op<N, OP, false>(p, r, k, op, e, gtid, gstride, io);
     else if (PROTO == kOneshotDB)
@@ -794,6 +898,8 @@ struct Row {
     t[N][kLLTwoshot][kAllgather] = nullptr;
     t[N][kSentinelTwoshot][kAllreduce] = reinterpret_cast<const void*>(&sfc_kernel<N, kSentinelTwoshot, kAllreduce>);
     t[N][kSentinelTwoshot][kAllgather] = nullptr;
+    t[N][kLL128Fast][kAllreduce] = reinterpret_cast<const void*>(&sfc_kernel<N, kLL128Fast, kAllreduce>);
+    t[N][kLL128Fast][kAllgather] = reinterpret_cast<const void*>(&sfc_kernel<N, kLL128Fast, kAllgather>);
   }
 };
 
@@ -823,7 +929,8 @@ uint64_t slot_bytes_gpu(int protocol, uint64_t count, int n) {
   switch (protocol) {
     case kLL:
       return ((nvec + kLLChunkVecs - 1) / kLLChunkVecs) * kLLChunkBytes;
-    case kLL128: {
+    case kLL128:
+    case kLL128Fast: {
       const uint64_t lines = (count + kLL128Elems - 1) / kLL128Elems;
       const uint64_t groups = (lines + kLL128LinesPerWarp - 1) / kLL128LinesPerWarp;
       return groups * kLL128LinesPerWarp * kLL128Line;

@@ -7,7 +7,6 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
-#include <mutex>
 #include <vector>
 
 #include "sfc.h"
@@ -67,7 +66,8 @@ bool cuda_ok(cudaError_t e) {
 }
 
 bool self_sync(int proto) {
-  return proto == kLL || proto == kLL128 || proto == kSentinel || proto == kLLTwoshot || proto == kSentinelTwoshot;
+  return proto == kLL || proto == kLL128 || proto == kSentinel || proto == kLLTwoshot || proto == kSentinelTwoshot ||
+         proto == kLL128Fast;
 }
 bool twoshot_alg(int proto) { return proto == kTwoshot || proto == kLLTwoshot || proto == kSentinelTwoshot; }
 
@@ -107,7 +107,7 @@ int choose_G(sfc_ctx* c, int proto, int op, uint64_t count, int* gmax_out) {
   if (c->cfg.ctas_per_rank > 0) return c->cfg.ctas_per_rank;
   const uint64_t nvec = (count + 7) / 8;
   uint64_t threads_needed;
-  if (proto == kLL128) {
+  if (proto == kLL128 || proto == kLL128Fast) {
     const uint64_t lines = (count + kLL128Elems - 1) / kLL128Elems;
     threads_needed = (lines + kLL128LinesPerWarp - 1) / kLL128LinesPerWarp * 32;
   } else if (twoshot_alg(proto)) {
@@ -249,8 +249,10 @@ void builtin_model(sfc_cost_model* m) {
           e.table_us[i] = pr < kCostProtocols ? kMeasuredP50Us[op][pr][n][i] : -1.0;
           measured = measured || e.table_us[i] > 0;
         }
-        // a protocol the sweep did not measure is never chosen by default
-        const bool exists = pr >= kLL && n >= kMinRanks && !(op == SFC_OP_ALLGATHER && twoshot_alg(pr));
+        // a protocol the sweep did not measure is never chosen by default, nor
+        // is the opt-in one-load LL128
+        const bool exists = pr >= kLL && pr != kLL128Fast && n >= kMinRanks &&
+                            !(op == SFC_OP_ALLGATHER && twoshot_alg(pr));
         e.alpha_us = exists && measured ? 0.0 : -1.0;
         e.beta_us_per_byte = 0.0;
       }
@@ -286,10 +288,12 @@ double sfc_algorithmic_bytes(sfc_op op, sfc_protocol protocol, size_t count, int
   switch (protocol) {
     case SFC_PROTO_LL:
     case SFC_PROTO_LL128:
+    case SFC_PROTO_LL128_FAST:
     case SFC_PROTO_SENTINEL: {
       double enc = s;
       if (protocol == SFC_PROTO_LL) enc = ll_enc(count);
-      if (protocol == SFC_PROTO_LL128) enc = 128.0 * static_cast<double>((count + kLL128Elems - 1) / kLL128Elems);
+      if (protocol == SFC_PROTO_LL128 || protocol == SFC_PROTO_LL128_FAST)
+        enc = 128.0 * static_cast<double>((count + kLL128Elems - 1) / kLL128Elems);
       const double reset = protocol == SFC_PROTO_SENTINEL ? (n - 1) * s : 0.0;
       const double written = op == SFC_OP_ALLREDUCE ? s : n * s;
       return n * (s + 2.0 * (n - 1) * enc + written + reset);
@@ -351,15 +355,16 @@ double sfc_cost_estimate(const sfc_cost_model* m, sfc_op op, sfc_protocol protoc
 }
 
 sfc_protocol sfc_select_protocol_model(const sfc_cost_model* m, sfc_op op, size_t bytes_per_rank, int nranks) {
-  static const int order[8] = {SFC_PROTO_SENTINEL,         SFC_PROTO_LL128,
-                               SFC_PROTO_LL,               SFC_PROTO_SENTINEL_TWOSHOT,
-                               SFC_PROTO_LL_TWOSHOT,       SFC_PROTO_BARRIER_ONESHOT_DB,
-                               SFC_PROTO_BARRIER_ONESHOT,  SFC_PROTO_BARRIER_TWOSHOT};
+  static const int order[9] = {SFC_PROTO_SENTINEL,         SFC_PROTO_LL128,
+                               SFC_PROTO_LL128_FAST,       SFC_PROTO_LL,
+                               SFC_PROTO_SENTINEL_TWOSHOT, SFC_PROTO_LL_TWOSHOT,
+                               SFC_PROTO_BARRIER_ONESHOT_DB, SFC_PROTO_BARRIER_ONESHOT,
+                               SFC_PROTO_BARRIER_TWOSHOT};
   if (m == nullptr || nranks < kMinRanks || nranks > kMaxRanks || (op != 0 && op != 1)) return SFC_PROTO_AUTO;
   const size_t count = bytes_per_rank / 2;
   int best = SFC_PROTO_AUTO;
   double best_t = 0, best_b = 0;
-  for (int i = 0; i < 8; ++i) {
+  for (int i = 0; i < 9; ++i) {
     const int pr = order[i];
     const double t = sfc_cost_estimate(m, op, static_cast<sfc_protocol>(pr), bytes_per_rank, nranks);
     if (t < 0) continue;
@@ -413,7 +418,7 @@ sfc_status sfc_init(sfc_ctx** out, int nranks, size_t max_bytes_per_rank, const 
   if (!cuda_ok(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, c->device)) || !coop)
     return fail(SFC_ERR_UNSUPPORTED);
   const uint64_t slots = static_cast<uint64_t>(nranks) * 2 * (nranks - 1);
-  for (int pr : {kLL, kLL128, kSentinel, kLLTwoshot, kSentinelTwoshot}) {
+  for (int pr : {kLL, kLL128, kSentinel, kLLTwoshot, kSentinelTwoshot, kLL128Fast}) {
     if (!provisioned(c, pr)) continue;
     const uint64_t sb = (slot_bytes_gpu(pr, c->max_count, nranks) + 255) / 256 * 256;
     c->slot_stride[pr] = sb;
@@ -465,7 +470,7 @@ sfc_status sfc_destroy(sfc_ctx* c) {
 sfc_status sfc_reset(sfc_ctx* c, void* stream) {
   if (c == nullptr) return SFC_ERR_INVALID;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  for (int pr : {kLL, kLL128, kSentinel, kLLTwoshot, kSentinelTwoshot}) {
+  for (int pr : {kLL, kLL128, kSentinel, kLLTwoshot, kSentinelTwoshot, kLL128Fast}) {
     if (c->region[pr] == nullptr) continue;
     const int fill = (pr == kSentinel || pr == kSentinelTwoshot) ? 0xFF : 0x00;
     if (!cuda_ok(cudaMemsetAsync(c->region[pr], fill, c->region_bytes[pr], st))) return SFC_ERR_CUDA;

@@ -16,7 +16,8 @@ the largest; with no measurements, alpha_p(N) + beta_p(N) * bytes_p(S, N)
 (the synchronization cost plus the transfer cost the flash-comm abstract
 weighs). The choice is the argmin; on a tie the protocol that moves fewer
 bytes wins, then the earlier one in the order
-sentinel < LL128 < LL < barrier oneshot < barrier twoshot.
+sentinel < LL128 < LL128 one-load < LL < sentinel twoshot < LL twoshot <
+dual-buffered oneshot < barrier oneshot < barrier twoshot.
 
 Which protocol wins where cannot be checked against the pages (they give no
 numbers): parity unpinned. The estimate and the argmin with its tie-break are
@@ -29,7 +30,7 @@ from . import protocols as P
 
 __all__ = ["TIE_ORDER", "algorithmic_bytes", "estimate", "choose"]
 
-TIE_ORDER = (P.SENTINEL, P.LL128, P.LL, "sentinel_twoshot", "ll_twoshot", "barrier_oneshot_db",
+TIE_ORDER = (P.SENTINEL, P.LL128, "ll128_fast", P.LL, "sentinel_twoshot", "ll_twoshot", "barrier_oneshot_db",
              "barrier_oneshot", "barrier_twoshot")
 
 
@@ -45,6 +46,8 @@ def algorithmic_bytes(proto, count, n, op="allreduce"):
     encoded shards, write N shards.
     """
     s = 2 * count
+    if proto == "ll128_fast":  # the LL128 layout, moved without fences
+        proto = P.LL128
     if proto in P.SELF_SYNC:
         enc = P.slot_bytes(proto, count)
         reset = (n - 1) * s if proto == P.SENTINEL else 0

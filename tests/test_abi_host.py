@@ -12,7 +12,7 @@ from oracle import selector as osel
 
 HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "sfc.h")
 PROTO_NAMES = {1: "ll", 2: "ll128", 3: "sentinel", 4: "barrier_oneshot", 5: "barrier_twoshot",
-               6: "barrier_oneshot_db", 7: "ll_twoshot", 8: "sentinel_twoshot"}
+               6: "barrier_oneshot_db", 7: "ll_twoshot", 8: "sentinel_twoshot", 9: "ll128_fast"}
 AR_ONLY = {5, 7, 8}
 
 
@@ -53,7 +53,7 @@ def _model_from(entries):
     """ctypes model from {proto: (alpha, beta, table)}; other protocols off."""
     m = api.default_cost_model()
     for op in range(2):
-        for p in range(9):
+        for p in range(10):
             for n in range(9):
                 m.c[op][p][n].alpha_us = -1.0
     for op in range(2):
@@ -110,5 +110,23 @@ def test_default_model_chooses_a_real_protocol_everywhere():
             for b in [512 << i for i in range(20)]:
                 p = api.select_protocol_model(m, op, b, n)
                 assert p != api.Protocol.AUTO
+                assert p != api.Protocol.LL128_FAST  # opt-in only
                 if op == "allgather":
                     assert int(p) not in AR_ONLY
+
+
+def test_one_load_ll128_is_opt_in():
+    """The built-in model carries the one-load LL128's measured latencies but
+    marks it unavailable; turning its entries on lets the selector take it
+    where it measured fastest (eight ranks, 64 KiB per rank)."""
+    m = api.default_cost_model()
+    op, n, b = "allreduce", 8, 64 << 10
+    e = m.c[int(api.as_op(op))][int(api.Protocol.LL128_FAST)][n]
+    assert e.alpha_us < 0 and e.table_us[16 - 9] > 0  # 2^16 bytes measured
+    assert api.cost_estimate(m, op, "ll128_fast", b, n) < 0
+    assert api.select_protocol_model(m, op, b, n) != api.Protocol.LL128_FAST
+    e.alpha_us = 0.0
+    t_fast = api.cost_estimate(m, op, "ll128_fast", b, n)
+    assert t_fast > 0
+    assert all(t_fast < api.cost_estimate(m, op, p, b, n) for p in ("ll", "ll128", "sentinel"))
+    assert api.select_protocol_model(m, op, b, n) == api.Protocol.LL128_FAST

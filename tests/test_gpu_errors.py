@@ -57,7 +57,7 @@ def test_bad_arguments_rejected():
 
 
 @pytest.mark.parametrize("proto", ["ll", "ll128", "sentinel", "barrier_oneshot", "barrier_twoshot",
-                                   "barrier_oneshot_db", "ll_twoshot", "sentinel_twoshot"])
+                                   "barrier_oneshot_db", "ll_twoshot", "sentinel_twoshot", "ll128_fast"])
 def test_silent_rank_times_out_and_recovers(proto):
     comm = api.Communicator(4, 1 << 14, timeout_us=2000)
     try:

@@ -20,8 +20,8 @@ from _gpu_helpers import Operands, run_chain, slot_bytes
 pytestmark = pytest.mark.gpu
 
 AR_PROTOS = ["ll", "ll128", "sentinel", "barrier_oneshot", "barrier_twoshot", "barrier_oneshot_db", "ll_twoshot",
-             "sentinel_twoshot"]
-AG_PROTOS = ["ll", "ll128", "sentinel", "barrier_oneshot", "barrier_oneshot_db"]
+             "sentinel_twoshot", "ll128_fast"]
+AG_PROTOS = ["ll", "ll128", "sentinel", "barrier_oneshot", "barrier_oneshot_db", "ll128_fast"]
 RAGGED = [1, 7, 8, 9, 59, 60, 61, 255, 1000, 4099]
 
 
@@ -229,7 +229,7 @@ def test_workload_decode_h8192_sentinel_full(tokens):
 
 
 @pytest.mark.parametrize("proto", ["ll128", "barrier_oneshot", "barrier_twoshot", "ll_twoshot", "sentinel_twoshot",
-                                   "barrier_oneshot_db"])
+                                   "barrier_oneshot_db", "ll128_fast"])
 @pytest.mark.parametrize("tokens", [1, 4, 16])
 def test_workload_decode_h4096_full(proto, tokens):
     """8 ranks, hidden 4096 x tokens, normal(0,0.5), 64 chained ops."""

@@ -49,7 +49,7 @@ def _run(proto, n, count, total_ops, skew_mean_ns, seed):
         comm.close()
 
 
-@pytest.mark.parametrize("proto", ["ll", "ll128", "sentinel", "ll_twoshot", "sentinel_twoshot"])
+@pytest.mark.parametrize("proto", ["ll", "ll128", "sentinel", "ll_twoshot", "sentinel_twoshot", "ll128_fast"])
 def test_million_ops_under_skew(proto):
     _run(proto, n=4, count=1000, total_ops=1_000_000, skew_mean_ns=300.0, seed=7)
 
@@ -57,3 +57,12 @@ def test_million_ops_under_skew(proto):
 @pytest.mark.parametrize("proto", ["ll", "sentinel", "barrier_oneshot", "barrier_oneshot_db", "barrier_twoshot"])
 def test_many_ops_eight_ranks(proto):
     _run(proto, n=8, count=4099, total_ops=1 << 17, skew_mean_ns=1000.0, seed=8)
+
+
+@pytest.mark.parametrize("n,count", [(2, 60), (8, 600), (4, 120000)])
+def test_ll128_one_load_tearing(n, count):
+    """The one-load LL128 accepts data read in the same warp load as its flag;
+    a torn line would show up here as a wrong element. Line-sized messages
+    (one line, ten lines) and a large one, every output checked."""
+    _run("ll128_fast", n=n, count=count, total_ops=1_000_000 if count < 100000 else 1 << 14,
+         skew_mean_ns=200.0, seed=9 + n)
