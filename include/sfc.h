@@ -301,12 +301,15 @@ sfc_status sfc_reserve_epochs(sfc_ctx* ctx, uint32_t k, uint32_t* first);
 /* Row-parallel linear layer fused with its all-reduce, for one decode token:
  * every rank r holds W[r] (bf16 [hidden][kdim], row-major: its slice of the
  * input dimension) and x[r] (bf16 [kdim]); the kernel computes the partial
- * p_r = bf16_RNE(W[r] x[r]) (fp32 accumulation) and, from the registers that
- * hold it, pushes it as LL units to every peer; each rank then polls,
- * reduces p_0..p_{N-1} in rank order in fp32 and writes y[r] (bf16
- * [hidden], identical on every rank). One launch, no intermediate buffer.
- * hidden % 8 == 0, hidden <= max count of the context; kdim % 8 == 0,
- * kdim <= 49152; all pointers 16-byte aligned; consumes one epoch. */
+ * p_r = bf16_RNE(W[r] x[r]) (fp32 accumulation) and pushes each finished
+ * 8-row vector of it as LL units to every peer while the rest of W[r] is
+ * still streaming; each rank then polls, reduces p_0..p_{N-1} in rank order
+ * in fp32 and writes y[r] (bf16 [hidden], identical on every rank). One
+ * cooperative launch (up to two CTAs per SM), no intermediate buffer in
+ * global memory. hidden % 8 == 0, hidden <= max count of the context;
+ * kdim % 8 == 0, kdim <= 49152; all pointers 16-byte aligned; consumes one
+ * epoch. SFC_ERR_RESOURCES if a CTA's shared memory (x[r], then 20 + 32 ks
+ * bytes per output vector it owns, ks <= 8) cannot fit. */
 sfc_status sfc_linear_allreduce(sfc_ctx* ctx, const void* const* W, const void* const* x, void* const* y,
                                 size_t hidden, size_t kdim, uint32_t epoch, void* stream);
 

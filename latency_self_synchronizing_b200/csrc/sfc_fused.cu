@@ -3,19 +3,25 @@
 // for Low-Latency LLM Inference", introduction, and "Why Microseconds Matter
 // in AI Infrastructure", section "Latency can matter more than bandwidth",
 // describe: per layer a sharded matrix product, then an all-reduce of the
-// activation). Built on the public device LL API (sfc_ll_device.cuh): the
-// partial product leaves the registers that computed it as LL units, with no
-// intermediate buffer and no second launch ("Why Microseconds Matter in AI
-// Infrastructure", section "Communication is becoming part of GPU execution").
+// activation). Built on the public device LL API (sfc_ll_device.cuh): each
+// finished 8-row output vector leaves as LL units while the weights of the
+// next ones are still streaming, with no intermediate buffer and no second
+// launch ("Why Microseconds Matter in AI Infrastructure", section
+// "Communication is becoming part of GPU execution").
 //
-// Rank r's CTAs compute p_r = W_r x_r: each warp owns output vectors (8 rows)
-// v = wg, wg + W, ... (W = warps per rank); for each it streams the 8 rows
-// of W_r once (lanes take consecutive 16-byte column chunks, fp32 FMA),
-// combines the lanes with a butterfly, rounds the 8 sums to bf16 and leaves
-// the vector in lane i for its i-th vector. Then every lane pushes its vector
-// to all peers and polls the peers' vectors for the same v (warp-collective,
-// bounded), folds them in rank order and stores y_r. The GEMV is HBM-bound
-// (weights are read once); no tensor cores.
+// Rank r owns G CTAs; CTA k owns the contiguous output vectors [v0, v1) of
+// p_r = W_r x_r (vector v = rows 8v .. 8v+7). The layer is bound by
+// streaming W from HBM once; a single token is a matrix-vector product, so
+// there is no tensor-core work. The CTA's 8 warps form 8 / ks groups of ks
+// warps; a group takes one vector at a time and its warps split the columns
+// into ks parts. A warp streams its 8 row segments with 16-byte loads
+// (lanes on consecutive chunks, 16 loads in flight per lane), keeps 8 fp32
+// dot products, and folds them across the warp in 9 shuffles (a transposing
+// butterfly: 4, 2, 1 values exchanged, then two plain levels), leaving row m's
+// sum in lanes 4m .. 4m+3. The last warp of a group to finish a vector adds
+// the ks parts in part order, rounds to bf16 and pushes the vector to every
+// peer. After the CTA's last vector, all its threads poll their vectors
+// (rank-order fp32 fold, one bf16 rounding) and store y_r.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -24,6 +30,15 @@
 
 namespace sfc {
 namespace {
+
+// streamed once: keep it out of L1
+SFC_DEV uint4 ld_stream_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
 
 SFC_DEV float dot8(uint4 w, uint4 x, float acc) {
   acc = fmaf(bf_lo(w.x), bf_lo(x.x), acc);
@@ -37,52 +52,98 @@ SFC_DEV float dot8(uint4 w, uint4 x, float acc) {
   return acc;
 }
 
+// Warp fold of 8 per-lane partial sums: returns the sum over all 32 lanes of
+// row m = 4 * bit4 + 2 * bit3 + bit2 of the lane index.
+SFC_DEV float fold8(const float (&a)[8], int lane) {
+  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+  float h[4], q[2];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float send = b4 ? a[i] : a[i + 4];
+    h[i] = (b4 ? a[i + 4] : a[i]) + __shfl_xor_sync(kFull, send, 16);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float send = b3 ? h[i] : h[i + 2];
+    q[i] = (b3 ? h[i + 2] : h[i]) + __shfl_xor_sync(kFull, send, 8);
+  }
+  float s = (b2 ? q[1] : q[0]) + __shfl_xor_sync(kFull, b2 ? q[0] : q[1], 4);
+  s += __shfl_xor_sync(kFull, s, 2);
+  s += __shfl_xor_sync(kFull, s, 1);
+  return s;
+}
+
+// Shared memory: x_r | parts [per][ks][8] fp32 | own [per] (packed bf16) |
+// counters [per].
 template <int NR>
-__global__ void __launch_bounds__(kLinearThreads, NR >= 6 ? 1 : 2) linear_allreduce_kernel(const __grid_constant__ LinearParams p) {
-  extern __shared__ uint4 xs[];  // x_r, kdim / 8 vectors
+__global__ void __launch_bounds__(kLinearThreads, 2) linear_allreduce_kernel(const __grid_constant__ LinearParams p) {
+  extern __shared__ __align__(16) unsigned char sm[];
   const int r = blockIdx.x / p.G;
   const int k = blockIdx.x - r * p.G;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint64_t kvec = p.kdim / 8;
-  const uint16_t* W = p.W[r];
+  const uint64_t kdim = p.kdim, kvec = kdim / 8, nvec = p.hidden / 8;
+  const uint32_t per = p.per_cta, ks = p.ks;
+  const uint64_t v0 = static_cast<uint64_t>(k) * per;
+  const uint64_t v1 = v0 + per < nvec ? v0 + per : nvec;
+  const uint32_t owned = v0 < v1 ? static_cast<uint32_t>(v1 - v0) : 0u;
+
+  uint4* xs = reinterpret_cast<uint4*>(sm);
+  float* parts = reinterpret_cast<float*>(sm + kdim * 2);
+  uint4* ownv = reinterpret_cast<uint4*>(parts + static_cast<uint64_t>(per) * ks * 8);
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(ownv + per);
+
   for (uint64_t i = threadIdx.x; i < kvec; i += blockDim.x) xs[i] = ld_nc_v4(p.x[r] + i * 8);
+  for (uint32_t i = threadIdx.x; i < per; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
-  const uint64_t nvec = p.hidden / 8;
-  const uint64_t wg = static_cast<uint64_t>(k) * (kLinearThreads / 32) + warp;
-  const uint64_t ws = static_cast<uint64_t>(p.G) * (kLinearThreads / 32);
-  for (uint64_t base = wg; base < nvec; base += ws * 32) {
-    uint4 mine = make_uint4(0, 0, 0, 0);
-    for (int i = 0; i < 32; ++i) {
-      const uint64_t v = base + static_cast<uint64_t>(i) * ws;
-      if (v >= nvec) break;  // warp-uniform
-      float acc[8];
+
+  const uint32_t groups = kLinearWarps / ks, g = warp / ks, h = warp % ks;
+  const uint64_t c_lo = kvec * h / ks, c_hi = kvec * (h + 1) / ks;  // this warp's column chunks
+  const uint16_t* W = p.W[r];
+  for (uint32_t t = g; t < owned; t += groups) {
+    const uint16_t* rows = W + (v0 + t) * 8 * kdim;
+    float acc[8];
 #pragma unroll
-      for (int m = 0; m < 8; ++m) acc[m] = 0.f;
-      const uint16_t* rows = W + v * 8 * p.kdim;
+    for (int m = 0; m < 8; ++m) acc[m] = 0.f;
 #pragma unroll 2
-      for (uint64_t c = lane; c < kvec; c += 32) {
-        const uint4 xv = xs[c];
-        uint4 wv[8];
+    for (uint64_t c = c_lo + lane; c < c_hi; c += 32) {
+      const uint4 xv = xs[c];
+      uint4 wv[8];
 #pragma unroll
-        for (int m = 0; m < 8; ++m) wv[m] = ld_nc_v4(rows + m * p.kdim + c * 8);
+      for (int m = 0; m < 8; ++m) wv[m] = ld_stream_v4(rows + m * kdim + c * 8);
 #pragma unroll
-        for (int m = 0; m < 8; ++m) acc[m] = dot8(wv[m], xv, acc[m]);
-      }
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc[m] += __shfl_xor_sync(kFull, acc[m], off);
-      }
-      if (lane == i)
-        mine = make_uint4(pack_rn(acc[0], acc[1]), pack_rn(acc[2], acc[3]), pack_rn(acc[4], acc[5]),
-                          pack_rn(acc[6], acc[7]));
+      for (int m = 0; m < 8; ++m) acc[m] = dot8(wv[m], xv, acc[m]);
     }
-    const uint64_t v = base + static_cast<uint64_t>(lane) * ws;
-    const bool act = v < nvec;
-    if (act) sfc_device::ll_push(p.view, r, p.epoch, v, mine);
+    const float s = fold8(acc, lane);
+    float* pt = parts + (static_cast<uint64_t>(t) * ks + h) * 8;
+    if ((lane & 3) == 0) pt[lane >> 2] = s;
+    __threadfence_block();
+    __syncwarp();
+    if (lane == 0) {
+      // the last of the group's ks warps completes the vector
+      if (atomicAdd(&cnt[t], 1u) == ks - 1) {
+        __threadfence_block();
+        const volatile float* pv = parts + static_cast<uint64_t>(t) * ks * 8;
+        float y[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          y[m] = pv[m];
+          for (uint32_t j = 1; j < ks; ++j) y[m] += pv[j * 8 + m];
+        }
+        const uint4 own = make_uint4(pack_rn(y[0], y[1]), pack_rn(y[2], y[3]), pack_rn(y[4], y[5]),
+                                     pack_rn(y[6], y[7]));
+        ownv[t] = own;
+        sfc_device::ll_push(p.view, r, p.epoch, v0 + t, own);
+      }
+    }
+  }
+  __syncthreads();  // every vector of the CTA is pushed and its own part stored
+  for (uint32_t base = 0; base < owned; base += kLinearThreads) {
+    const uint32_t t = base + threadIdx.x;
+    const bool act = t < owned;
+    const uint4 own = act ? ownv[t] : make_uint4(0, 0, 0, 0);
     uint4 out;
-    if (!sfc_device::ll_allreduce_lane<NR>(p.view, r, p.epoch, v, act, mine, &out)) return;
-    if (act) *reinterpret_cast<uint4*>(p.y[r] + v * 8) = out;
+    if (!sfc_device::ll_allreduce_lane<NR>(p.view, r, p.epoch, v0 + t, act, own, &out)) return;
+    if (act) *reinterpret_cast<uint4*>(p.y[r] + (v0 + t) * 8) = out;
   }
 }
 

@@ -101,9 +101,16 @@ struct LinearParams {
   uint64_t kdim;
   int G;                         // CTAs per rank
   uint32_t epoch;
+  uint32_t per_cta;              // output vectors per CTA
+  uint32_t ks;                   // warps that split one vector's columns (1, 2, 4 or 8)
   sfc_ll_view view;
 };
 constexpr int kLinearThreads = 256;
+constexpr int kLinearWarps = kLinearThreads / 32;
+// dynamic shared memory of the fused kernel: x, per-part sums, own vectors, counters
+inline size_t linear_smem_bytes(uint64_t kdim, uint32_t ks, uint32_t per_cta) {
+  return kdim * 2 + 32ull * ks * per_cta + 16ull * per_cta + 4ull * per_cta;
+}
 const void* linear_kernel_for(int nranks);
 
 // Kernel entry for (nranks, protocol, op); null if not provided.

@@ -42,6 +42,8 @@ struct sfc_ctx {
   sfc_cost_model model{};
 
   int occupancy[kNumProtocols][2] = {};  // blocks per SM, per (protocol, op), 0 = unknown
+  int smem_optin = 0;                     // opt-in shared memory per block (bytes)
+  int linear_occ = 0;                     // fused-linear CTAs per SM (0 = not yet queried)
 
   // staging for the host-buffer entry point
   uint16_t* stage_in = nullptr;
@@ -414,6 +416,8 @@ sfc_status sfc_init(sfc_ctx** out, int nranks, size_t max_bytes_per_rank, const 
   if (!cuda_ok(cudaGetDevice(&c->device))) return fail(SFC_ERR_CUDA);
   if (!cuda_ok(cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, c->device)))
     return fail(SFC_ERR_CUDA);
+  if (!cuda_ok(cudaDeviceGetAttribute(&c->smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, c->device)))
+    return fail(SFC_ERR_CUDA);
   int coop = 0;
   if (!cuda_ok(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, c->device)) || !coop)
     return fail(SFC_ERR_UNSUPPORTED);
@@ -649,19 +653,43 @@ sfc_status sfc_linear_allreduce(sfc_ctx* c, const void* const* W, const void* co
           (a < b && overlap(y[a], hidden * 2, y[b], hidden * 2)))
         return SFC_ERR_INVALID;
   const void* fn = linear_kernel_for(N);
-  const int smem = static_cast<int>(kdim * 2);
-  if (smem > 48 * 1024 &&
-      !cuda_ok(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
-    return SFC_ERR_CUDA;
-  int occ = 0;
-  if (!cuda_ok(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kLinearThreads, smem)) || occ < 1)
-    return SFC_ERR_RESOURCES;
-  // every SM streams weights: as many CTAs per rank as can be co-resident,
-  // but no more warps than output vectors
-  const int gmax = occ * c->sm_count / N;
-  const uint64_t warps_needed = (hidden / 8);
-  const int G = static_cast<int>(std::min<uint64_t>(gmax, (warps_needed + 7) / 8));
-  if (G < 1) return SFC_ERR_RESOURCES;
+  // as many CTAs per rank as fit (two per SM), each rank's output vectors
+  // split evenly over its CTAs; ks warps share a vector when that evens out
+  // the 8 warps' work (every part keeps at least 128 column chunks, four per
+  // lane)
+  const uint64_t nvec = hidden / 8, kvec = kdim / 8;
+  int occ = c->linear_occ;
+  if (occ == 0) {
+    if (!cuda_ok(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, c->smem_optin)))
+      return SFC_ERR_CUDA;
+    if (!cuda_ok(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kLinearThreads, 0)) || occ < 1)
+      return SFC_ERR_RESOURCES;
+    c->linear_occ = occ = std::min(occ, 2);
+  }
+  int G = occ * c->sm_count / N;
+  uint32_t per = 0, ks = 1;
+  for (;; --G) {
+    if (G < 1) return SFC_ERR_RESOURCES;
+    per = static_cast<uint32_t>((nvec + G - 1) / G);
+    double best = -1.0;
+    for (uint32_t cand = 1; cand <= 8; cand *= 2) {
+      if (cand > 1 && kvec / cand < 128) break;
+      const uint32_t groups = 8 / cand, rounds = (per + groups - 1) / groups;
+      const double eff = static_cast<double>(per) / (static_cast<double>(rounds) * groups);
+      if (eff > best + 1e-9) {
+        best = eff;
+        ks = cand;
+      }
+    }
+    // both CTAs of an SM must fit: fewer, larger CTAs if not
+    const size_t smem = sfc::linear_smem_bytes(kdim, ks, per);
+    if (smem <= static_cast<size_t>(c->smem_optin) &&
+        (G * N <= c->sm_count || 2 * (smem + 1024) <= static_cast<size_t>(c->smem_optin) + 1024))
+      break;
+  }
+  const int smem = static_cast<int>(sfc::linear_smem_bytes(kdim, ks, per));
+  p.per_cta = per;
+  p.ks = ks;
   p.hidden = hidden;
   p.kdim = kdim;
   p.G = G;

@@ -7,10 +7,12 @@ pair (a batched matrix-vector product for all ranks, then an all-reduce).
 Shapes default to a Llama-3.1-70B MLP down projection with 4-way tensor
 parallelism (hidden 8192, intermediate 28672 / 4 = 7168 per rank), one
 decode token. Weights are normal(0, 0.05), drawn on the device by torch's
-seeded generator (timing only; parity is the tests' job). The weights of all
-ranks (N * hidden * kdim * 2 bytes) exceed L2, so every iteration reads them
-from HBM. Prints one JSON line: microseconds per layer for both, and the
-fused kernel's weight-streaming bandwidth against the measured HBM copy
+seeded generator (timing only; parity is the tests' job). Consecutive calls
+use different copies of the weights (at least 320 MB in all), so no call
+finds its weights in L2 and every call streams them from HBM. Time per
+layer = mean over `iters` back-to-back calls between two CUDA events (median
+of 5 such runs). Prints one JSON line: microseconds per layer for both, and
+the fused kernel's weight-streaming bandwidth against the measured HBM copy
 bandwidth.
 """
 
@@ -24,18 +26,22 @@ import torch
 from . import api
 
 
-def _events(fn, iters, warmup=5):
+def _events(fn, iters, reps=5, warmup=5):
+    """Median over `reps` of the mean time per call of `iters` back-to-back
+    calls between two events (a decode step issues its layers back to back,
+    so host-side call overhead overlaps the previous layer's GPU time)."""
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
     times = []
-    for _ in range(iters):
+    for _ in range(reps):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        fn()
+        for _ in range(iters):
+            fn()
         b.record()
         torch.cuda.synchronize()
-        times.append(a.elapsed_time(b) * 1e3)
+        times.append(a.elapsed_time(b) * 1e3 / iters)
     return statistics.median(times)
 
 
@@ -50,23 +56,30 @@ def main(argv=None):
     dev = torch.device("cuda")
     gen = torch.Generator(device=dev)
     gen.manual_seed(0)
-    w = (torch.randn(n, hidden, kdim, generator=gen, device=dev) * 0.05).to(torch.bfloat16)
+    wbytes = n * hidden * kdim * 2
+    # enough weight copies, used in turn, that consecutive layers never find
+    # their weights in the 126 MB L2 (a decode step's layers are distinct)
+    copies = max(2, -(-(320 << 20) // wbytes))
+    ws = [(torch.randn(n, hidden, kdim, generator=gen, device=dev) * 0.05).to(torch.bfloat16) for _ in range(copies)]
     x = torch.randn(n, kdim, 1, generator=gen, device=dev).to(torch.bfloat16)
     y = torch.empty(n, hidden, dtype=torch.bfloat16, device=dev)
     part = torch.empty(n, hidden, 1, dtype=torch.bfloat16, device=dev)
     y2 = torch.empty(n, hidden, dtype=torch.bfloat16, device=dev)
     comm = api.Communicator(n, hidden * 2)
-    W = [w[r] for r in range(n)]
+    Ws = [[w[r] for r in range(n)] for w in ws]
     X = [x[r, :, 0] for r in range(n)]
     Y = [y[r] for r in range(n)]
     P = [part[r, :, 0] for r in range(n)]
     Y2 = [y2[r] for r in range(n)]
+    turn = [0]
 
     def fused():
-        comm.linear_allreduce(W, X, Y)
+        turn[0] = (turn[0] + 1) % copies
+        comm.linear_allreduce(Ws[turn[0]], X, Y)
 
     def unfused():
-        torch.bmm(w, x, out=part)
+        turn[0] = (turn[0] + 1) % copies
+        torch.bmm(ws[turn[0]], x, out=part)
         comm.allreduce(P, Y2, protocol="auto")
 
     t_f = _events(fused, a.iters)
@@ -80,8 +93,8 @@ def main(argv=None):
                                                  "MEASURED_PEAKS.json")))["hbm_gbs"])
     except (OSError, KeyError, ValueError):
         pass
-    wbytes = n * hidden * kdim * 2
-    print(json.dumps({"nranks": n, "hidden": hidden, "kdim": kdim, "fused_us": t_f, "unfused_us": t_u,
+    print(json.dumps({"nranks": n, "hidden": hidden, "kdim": kdim, "weight_copies": copies, "fused_us": t_f,
+                      "unfused_us": t_u,
                       "unfused_selected_protocol": comm.select_protocol("allreduce", hidden * 2).name.lower(),
                       "fused_weight_gbs": wbytes / (t_f * 1e-6) / 1e9, "hbm_peak_gbs": peak,
                       "fused_frac": wbytes / (t_f * 1e-6) / 1e9 / peak}))
