@@ -248,7 +248,9 @@ const char* sfc_status_string(sfc_status s);
 /* The epoch the next operation must use. */
 uint32_t sfc_next_epoch(const sfc_ctx* ctx);
 
-/* The launch shape a call would use: CTAs per rank and threads per CTA. */
+/* The launch shape a call would use: CTAs per rank and threads per CTA
+ * (256, or 128 for LL, sentinel and one-load LL128 messages of at most
+ * 64 KB per rank at 4 or more ranks when ctas_per_rank is 0). */
 sfc_status sfc_launch_shape(sfc_ctx* ctx, sfc_op op, sfc_protocol protocol, size_t count,
                             int* ctas_per_rank, int* threads_per_cta);
 

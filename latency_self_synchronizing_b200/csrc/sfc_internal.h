@@ -10,7 +10,9 @@
 
 namespace sfc {
 
-constexpr int kThreads = 256;  // threads per CTA of every collective kernel
+constexpr int kThreads = 256;  // threads per CTA of the collective kernels (launch bound)
+constexpr int kSmallCtaThreads = 128;      // CTA size for small messages at 4+ ranks
+constexpr uint64_t kSmallCtaMaxCount = 32768;  // bf16 per rank (64 KB) up to which it applies
 constexpr int kMaxRanks = 8;
 constexpr int kMinRanks = 2;
 

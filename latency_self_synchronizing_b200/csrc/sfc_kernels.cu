@@ -838,8 +838,9 @@ template <int N, int PROTO, int OP>
 __global__ void __launch_bounds__(kThreads, MinBlocks<N, PROTO>::value) sfc_kernel(const __grid_constant__ KParams p) {
   const int r = blockIdx.x / p.G;
   const int k = blockIdx.x - r * p.G;
-  const uint64_t gtid = static_cast<uint64_t>(k) * kThreads + threadIdx.x;
-  const uint64_t gstride = static_cast<uint64_t>(p.G) * kThreads;
+  // the launch picks 128 or kThreads threads per CTA; every rank uses the same
+  const uint64_t gtid = static_cast<uint64_t>(k) * blockDim.x + threadIdx.x;
+  const uint64_t gstride = static_cast<uint64_t>(p.G) * blockDim.x;
   const int lane = threadIdx.x & 31;
   if (ld_rlx_s32(&p.status->abort)) return;  // poisoned context: do nothing
   if (p.timings != nullptr && lane == 0)

@@ -130,3 +130,4 @@ def test_one_load_ll128_is_opt_in():
     assert t_fast > 0
     assert all(t_fast < api.cost_estimate(m, op, p, b, n) for p in ("ll", "ll128", "sentinel"))
     assert api.select_protocol_model(m, op, b, n) == api.Protocol.LL128_FAST
+

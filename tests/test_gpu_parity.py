@@ -305,3 +305,18 @@ def test_guard_words_intact_after_large_chain(proto):
         assert comm.check_guards() == api.Status.OK
     finally:
         comm.close()
+
+
+@pytest.mark.parametrize("proto", ["ll", "sentinel", "ll128_fast"])
+@pytest.mark.parametrize("n", [4, 8])
+def test_cta_size_boundary(comms, proto, n):
+    """Messages up to 64 KB per rank at 4+ ranks run in 128-thread CTAs, larger
+    ones in 256-thread CTAs; both sides of the boundary are bit-exact and both
+    op kinds share one context and epoch sequence."""
+    comm = comms(n, 1 << 17)
+    for count, threads in [(32768, 128), (32769, 256), (8191, 128)]:
+        assert comm.launch_shape("allreduce", proto, count)[1] == threads
+        x = make_inputs(seed=count + n, k_ops=3, nranks=n, count=count)
+        _assert_ar(run_chain(comm, proto, x), x)
+        xg = make_inputs(seed=count + n + 1, k_ops=2, nranks=n, count=count // n)
+        _assert_ag(run_chain(comm, proto, xg, op="allgather"), xg)
