@@ -349,13 +349,14 @@ def run_gpu(args):
 def kernel_sources_sha():
     """SHA-256 over the sources that decide what the chain kernels do and how
     they are launched (kernels, device helpers, internal header, runtime); the
-    selector's measured table, the floor benchmark and the allocation-free
-    entry point do not change a chain launch and are left out."""
+    selector's measured table, the floor benchmark, the allocation-free
+    entry point and the fused linear kernel do not change a chain launch and
+    are left out."""
     import hashlib
 
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "latency_self_synchronizing_b200", "csrc")
-    skip = ("sfc_cost_table.h", "sfc_floor.cu", "sfc_noalloc.cu")
+    skip = ("sfc_cost_table.h", "sfc_floor.cu", "sfc_noalloc.cu", "sfc_fused.cu")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh", ".h")) and name not in skip:
             h.update(name.encode())

@@ -79,10 +79,14 @@ def measure_point(comm, op, proto, count, k_ops, reps, gen, dev):
 
 
 def evaluate_selector(points, model):
-    """Per swept (op, N, size): the model's choice vs the measured fastest."""
+    """Per swept (op, N, size): the model's choice vs the measured fastest of
+    the protocols the model may choose (an opt-in protocol the model marks
+    unavailable is not a candidate)."""
     best = {}
     for p in points:
         key = (p["op"], p["nranks"], p["bytes_per_rank"])
+        if api.cost_estimate(model, p["op"], p["protocol"], p["bytes_per_rank"], p["nranks"]) < 0:
+            continue
         if key not in best or p["p50_us"] < best[key]["p50_us"]:
             best[key] = p
     rows = []
@@ -103,7 +107,7 @@ def main(argv=None):
     ap.add_argument("--op", default="allreduce", choices=["allreduce", "allgather"])
     ap.add_argument("--protocols", nargs="+",
                     default=["ll", "ll128", "sentinel", "barrier_oneshot", "barrier_twoshot", "barrier_oneshot_db",
-                             "ll_twoshot", "sentinel_twoshot"])
+                             "ll_twoshot", "sentinel_twoshot", "ll128_fast"])
     ap.add_argument("--min-bytes", type=int, default=1024)
     ap.add_argument("--max-bytes", type=int, default=64 << 20)
     ap.add_argument("--k-ops", type=int, default=50)
