@@ -199,9 +199,14 @@ sfc_status sfc_allgather_chain(sfc_ctx* ctx, int k_ops, const void* const* in_ta
 /* End-to-end all-reduce chain from HOST memory: in_host holds
  * [k_ops][N][count] bf16 contiguous, out_host receives [k_ops][N][count].
  * Copies the inputs to context-owned device staging (allocated on first use,
- * grown as needed), runs the chain, copies the outputs back, all on
- * `stream`; the call returns once the copies are queued. Page-locked host
- * memory makes the copies asynchronous. timings as in sfc_allreduce_chain. */
+ * grown as needed; growing waits for the device), runs the chain, copies the
+ * outputs back. The chain runs as up to 8 launches of at least 16
+ * operations, and the copies of one segment overlap the run of its
+ * neighbours on two context-owned copy streams; events tie them to
+ * `stream`, which ends up waiting for the last copy, so the call is ordered
+ * on `stream` like any other. It returns once everything is queued.
+ * Page-locked host memory makes the copies asynchronous. timings as in
+ * sfc_allreduce_chain. */
 sfc_status sfc_allreduce_chain_host(sfc_ctx* ctx, int k_ops, const void* in_host, void* out_host,
                                     size_t count, sfc_dtype dtype, sfc_protocol protocol,
                                     uint32_t first_epoch, uint64_t* timings, void* stream);

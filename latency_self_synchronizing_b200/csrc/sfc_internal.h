@@ -11,6 +11,8 @@
 namespace sfc {
 
 constexpr int kThreads = 256;  // threads per CTA of the collective kernels (launch bound)
+constexpr int kHostSegmentsMax = 8;    // host-buffer chains: launches whose copies overlap
+constexpr int kHostSegmentMinOps = 16;  // fewest operations per such launch
 constexpr int kSmallCtaThreads = 128;      // CTA size for small messages at 4+ ranks
 constexpr uint64_t kSmallCtaMaxCount = 32768;  // bf16 per rank (64 KB) up to which it applies
 constexpr int kMaxRanks = 8;
@@ -87,7 +89,8 @@ struct KParams {
   uint64_t red_stride;  // elements
 
   DevStatus* status;
-  uint64_t* timings;    // [k_ops + 1] or null
+  uint64_t* timings;    // [timing_first + k_ops + 1] or null
+  uint32_t timing_first;  // completion of op k is stamped at timings[1 + timing_first + k]
   const uint32_t* skew; // [k_ops * N] ns or null
   uint64_t timeout_ns;
   int debug;

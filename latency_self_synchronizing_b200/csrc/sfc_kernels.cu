@@ -874,7 +874,8 @@ __global__ void __launch_bounds__(kThreads, MinBlocks<N, PROTO>::value) sfc_kern
     io.in = io.in_next;
     io.out = out_next;
     if (p.timings != nullptr && lane == 0)
-      atomicMax(reinterpret_cast<unsigned long long*>(&p.timings[1 + op]), static_cast<unsigned long long>(gtimer()));
+      atomicMax(reinterpret_cast<unsigned long long*>(&p.timings[1 + p.timing_first + op]),
+                static_cast<unsigned long long>(gtimer()));
   }
 }
 

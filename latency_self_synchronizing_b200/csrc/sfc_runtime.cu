@@ -45,10 +45,14 @@ struct sfc_ctx {
   int smem_optin = 0;                     // opt-in shared memory per block (bytes)
   int linear_occ = 0;                     // fused-linear CTAs per SM (0 = not yet queried)
 
-  // staging for the host-buffer entry point
+  // staging for the host-buffer entry point, and the copy streams and
+  // events that overlap its copies with the chain segments
   uint16_t* stage_in = nullptr;
   uint16_t* stage_out = nullptr;
   size_t stage_bytes = 0;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t ev_start = nullptr;
+  cudaEvent_t ev_in[kHostSegmentsMax] = {}, ev_run[kHostSegmentsMax] = {}, ev_out[kHostSegmentsMax] = {};
 };
 
 namespace {
@@ -479,6 +483,12 @@ sfc_status sfc_destroy(sfc_ctx* c) {
   if (c->hstatus) cudaFreeHost(c->hstatus);
   if (c->stage_in) cudaFree(c->stage_in);
   if (c->stage_out) cudaFree(c->stage_out);
+  if (c->h2d) cudaStreamDestroy(c->h2d);
+  if (c->d2h) cudaStreamDestroy(c->d2h);
+  if (c->ev_start) cudaEventDestroy(c->ev_start);
+  for (int i = 0; i < kHostSegmentsMax; ++i)
+    for (cudaEvent_t ev : {c->ev_in[i], c->ev_run[i], c->ev_out[i]})
+      if (ev) cudaEventDestroy(ev);
   delete c;
   return SFC_OK;
 }
@@ -537,7 +547,8 @@ sfc_status sfc_allreduce_chain_host(sfc_ctx* c, int k_ops, const void* in_host, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (need > c->stage_bytes) {
     if (c->stage_in || c->stage_out) {
-      if (!cuda_ok(cudaStreamSynchronize(st))) return SFC_ERR_CUDA;
+      // every earlier copy was joined into the caller's stream it was issued on
+      if (!cuda_ok(cudaDeviceSynchronize())) return SFC_ERR_CUDA;
       cudaFree(c->stage_in);
       cudaFree(c->stage_out);
       c->stage_in = c->stage_out = nullptr;
@@ -546,27 +557,75 @@ sfc_status sfc_allreduce_chain_host(sfc_ctx* c, int k_ops, const void* in_host, 
     if (!cuda_ok(cudaMalloc(&c->stage_in, need)) || !cuda_ok(cudaMalloc(&c->stage_out, need))) return SFC_ERR_CUDA;
     c->stage_bytes = need;
   }
-  const size_t rows = static_cast<size_t>(k_ops) * c->nranks;
-  if (!cuda_ok(cudaMemcpy2DAsync(c->stage_in, stride * 2, in_host, count * 2, count * 2, rows,
-                                 cudaMemcpyHostToDevice, st)))
-    return SFC_ERR_CUDA;
+  if (c->h2d == nullptr) {
+    if (!cuda_ok(cudaStreamCreateWithFlags(&c->h2d, cudaStreamNonBlocking)) ||
+        !cuda_ok(cudaStreamCreateWithFlags(&c->d2h, cudaStreamNonBlocking)) ||
+        !cuda_ok(cudaEventCreateWithFlags(&c->ev_start, cudaEventDisableTiming)))
+      return SFC_ERR_CUDA;
+    for (int i = 0; i < kHostSegmentsMax; ++i)
+      if (!cuda_ok(cudaEventCreateWithFlags(&c->ev_in[i], cudaEventDisableTiming)) ||
+          !cuda_ok(cudaEventCreateWithFlags(&c->ev_run[i], cudaEventDisableTiming)) ||
+          !cuda_ok(cudaEventCreateWithFlags(&c->ev_out[i], cudaEventDisableTiming)))
+        return SFC_ERR_CUDA;
+  }
   s = prepare_timings(timings, k_ops, st);
   if (s != SFC_OK) return s;
-  KParams p{};
-  p.addr_mode = 2;
-  p.in_base = c->stage_in;
-  p.out_base = c->stage_out;
-  p.in_stride = stride;
-  p.out_stride = stride;
-  p.timings = timings;
   const int G = choose_G(c, proto, SFC_OP_ALLREDUCE, count, nullptr);
-  fill_common(c, p, proto, count, k_ops, first_epoch, G);
-  s = launch(c, proto, SFC_OP_ALLREDUCE, p, st);
-  if (s != SFC_OK) return s;
-  c->next_epoch = first_epoch + static_cast<uint32_t>(k_ops);
-  if (!cuda_ok(cudaMemcpy2DAsync(out_host, count * 2, c->stage_out, stride * 2, count * 2, rows,
-                                 cudaMemcpyDeviceToHost, st)))
+  // The chain runs as `nseg` consecutive launches of consecutive operations.
+  // All input copies are queued first on the h2d stream (a cooperative
+  // launch can hold the host until the device starts it, so queuing them
+  // between launches would delay them); segment j waits only for its own
+  // inputs, and its outputs are copied out on the d2h stream while segment
+  // j+1 runs. The caller's stream finally waits for the last output copy, so
+  // the call is ordered on `stream` like any other.
+  const int nseg = std::max(1, std::min(kHostSegmentsMax, k_ops / kHostSegmentMinOps));
+  const size_t row_dev = stride * 2, row_host = count * 2;
+  auto seg_rows = [&](int j, size_t* row0, size_t* rows) {
+    const int64_t a = static_cast<int64_t>(k_ops) * j / nseg, b = static_cast<int64_t>(k_ops) * (j + 1) / nseg;
+    *row0 = static_cast<size_t>(a) * c->nranks;
+    *rows = static_cast<size_t>(b - a) * c->nranks;
+    return static_cast<int>(a);
+  };
+  // one flat copy when host and device rows have the same pitch
+  auto copy = [&](void* dst, size_t dpitch, const void* src, size_t spitch, size_t rows, cudaMemcpyKind kind,
+                  cudaStream_t cs) {
+    if (dpitch == spitch) return cuda_ok(cudaMemcpyAsync(dst, src, rows * row_host, kind, cs));
+    return cuda_ok(cudaMemcpy2DAsync(dst, dpitch, src, spitch, row_host, rows, kind, cs));
+  };
+  if (!cuda_ok(cudaEventRecord(c->ev_start, st)) || !cuda_ok(cudaStreamWaitEvent(c->h2d, c->ev_start, 0)))
     return SFC_ERR_CUDA;
+  for (int j = 0; j < nseg; ++j) {
+    size_t row0, rows;
+    (void)seg_rows(j, &row0, &rows);
+    if (!copy(c->stage_in + row0 * stride, row_dev, static_cast<const uint8_t*>(in_host) + row0 * row_host, row_host,
+              rows, cudaMemcpyHostToDevice, c->h2d) ||
+        !cuda_ok(cudaEventRecord(c->ev_in[j], c->h2d)))
+      return SFC_ERR_CUDA;
+  }
+  for (int j = 0; j < nseg; ++j) {
+    size_t row0, rows;
+    const int a = seg_rows(j, &row0, &rows);
+    const int kj = static_cast<int>(rows / c->nranks);
+    if (!cuda_ok(cudaStreamWaitEvent(st, c->ev_in[j], 0))) return SFC_ERR_CUDA;
+    KParams p{};
+    p.addr_mode = 2;
+    p.in_base = c->stage_in + row0 * stride;
+    p.out_base = c->stage_out + row0 * stride;
+    p.in_stride = stride;
+    p.out_stride = stride;
+    p.timings = timings;
+    p.timing_first = static_cast<uint32_t>(a);
+    fill_common(c, p, proto, count, kj, first_epoch + static_cast<uint32_t>(a), G);
+    s = launch(c, proto, SFC_OP_ALLREDUCE, p, st);
+    if (s != SFC_OK) return s;
+    c->next_epoch = first_epoch + static_cast<uint32_t>(a + kj);
+    if (!cuda_ok(cudaEventRecord(c->ev_run[j], st)) || !cuda_ok(cudaStreamWaitEvent(c->d2h, c->ev_run[j], 0)) ||
+        !copy(static_cast<uint8_t*>(out_host) + row0 * row_host, row_host, c->stage_out + row0 * stride, row_dev,
+              rows, cudaMemcpyDeviceToHost, c->d2h) ||
+        !cuda_ok(cudaEventRecord(c->ev_out[j], c->d2h)))
+      return SFC_ERR_CUDA;
+  }
+  if (!cuda_ok(cudaStreamWaitEvent(st, c->ev_out[nseg - 1], 0))) return SFC_ERR_CUDA;
   return SFC_OK;
 }
 
