@@ -32,7 +32,8 @@ def _case(n, hidden, kdim, seed):
 
 # shapes cover every column split the launch picks (ks = 1, 2, 4, 8 warps per vector)
 @pytest.mark.parametrize("n,hidden,kdim", [(2, 8, 8), (2, 1000, 512), (4, 8192, 7168), (8, 4096, 1024),
-                                           (2, 64, 8192), (6, 1536, 4096), (3, 2056, 136), (8, 24, 8)])
+                                           (2, 64, 8192), (6, 1536, 4096), (3, 2056, 136), (8, 24, 8),
+                                           (5, 2048, 1024), (7, 1536, 2048)])
 def test_linear_allreduce_within_bound(n, hidden, kdim):
     w, x = _case(n, hidden, kdim, seed=hidden + kdim + n)
     comm = api.Communicator(n, hidden * 2, protocols=["ll"])

@@ -58,7 +58,7 @@ def comms():
 
 
 @pytest.mark.parametrize("proto", AR_PROTOS)
-@pytest.mark.parametrize("n", [2, 3, 4, 5, 8])
+@pytest.mark.parametrize("n", [2, 3, 4, 5, 6, 7, 8])
 def test_allreduce_ragged_chain(comms, proto, n):
     comm = comms(n)
     for i, count in enumerate(RAGGED):
@@ -67,7 +67,7 @@ def test_allreduce_ragged_chain(comms, proto, n):
 
 
 @pytest.mark.parametrize("proto", AG_PROTOS)
-@pytest.mark.parametrize("n", [2, 3, 8])
+@pytest.mark.parametrize("n", [2, 3, 4, 5, 6, 7, 8])
 def test_allgather_ragged_chain(comms, proto, n):
     comm = comms(n)
     for i, count in enumerate([1, 7, 8, 61, 1000, 4099]):

@@ -66,3 +66,11 @@ def test_ll128_one_load_tearing(n, count):
     (one line, ten lines) and a large one, every output checked."""
     _run("ll128_fast", n=n, count=count, total_ops=1_000_000 if count < 100000 else 1 << 14,
          skew_mean_ns=200.0, seed=9 + n)
+
+
+@pytest.mark.parametrize("proto", ["ll", "sentinel", "ll128_fast", "ll_twoshot", "sentinel_twoshot", "barrier_oneshot_db"])
+@pytest.mark.parametrize("n", [3, 5, 6, 7])
+def test_odd_rank_counts_under_skew(proto, n):
+    """Rank counts the power-of-two cases do not reach (uneven twoshot shards,
+    source indices that skip the own rank at every position), ragged size."""
+    _run(proto, n=n, count=777, total_ops=1 << 15, skew_mean_ns=500.0, seed=20 + n)
