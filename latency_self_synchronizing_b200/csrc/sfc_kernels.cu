@@ -752,6 +752,17 @@ SFC_DEV bool cta_barrier(const KParams& p, int r, int k, int op, uint64_t target
 // All-Reduce for Low-Latency LLM Inference", abstract). The dual-buffered
 // variant drops the bottom barrier: the caller alternates two input buffers,
 // which is SiFAR's co-design of communication and model execution.
+// Oneshot result for vector v: the rank-order reduction, or the N copies.
+template <int N, int OP>
+SFC_DEV void oneshot_emit(uint16_t* out_r, uint64_t v, const uint4 (&x)[N], uint64_t count) {
+  if (OP == kAllreduce) {
+    store_n(out_r, v * 8, reduce8<N>(x), 8, count);
+  } else {
+#pragma unroll
+    for (int q = 0; q < N; ++q) store_n(out_r, q * count + v * 8, x[q], 8, q * count + count);
+  }
+}
+
 template <int N, int OP, bool kDualBuffered>
 SFC_DEV bool oneshot_op(const KParams& p, int r, int k, int op, uint32_t e, uint64_t gtid, uint64_t gstride,
                         const Operands& io) {
@@ -764,16 +775,24 @@ SFC_DEV bool oneshot_op(const KParams& p, int r, int k, int op, uint32_t e, uint
   const uint16_t* src[N];
 #pragma unroll
   for (int q = 0; q < N; ++q) src[q] = in_ptr<N>(p, op, q);
-  for (uint64_t v = gtid; v < nvec; v += gstride) {
+  // U of the thread's vectors per step (U * N loads in flight before any
+  // use) while U remain, then one at a time
+  constexpr int U = N <= 2 ? 4 : 2;
+  uint64_t v = gtid;
+  for (; v + (U - 1) * gstride < nvec; v += U * gstride) {
+    uint4 x[U][N];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int q = 0; q < N; ++q) x[u][q] = load8(src[q], (v + u * gstride) * 8, count);
+#pragma unroll
+    for (int u = 0; u < U; ++u) oneshot_emit<N, OP>(out_r, v + u * gstride, x[u], count);
+  }
+  for (; v < nvec; v += gstride) {
     uint4 x[N];
 #pragma unroll
     for (int q = 0; q < N; ++q) x[q] = load8(src[q], v * 8, count);
-    if (OP == kAllreduce) {
-      store_n(out_r, v * 8, reduce8<N>(x), 8, count);
-    } else {
-#pragma unroll
-      for (int q = 0; q < N; ++q) store_n(out_r, q * count + v * 8, x[q], 8, q * count + count);
-    }
+    oneshot_emit<N, OP>(out_r, v, x, count);
   }
   // with dual-buffered inputs the next operation's top barrier already
   // orders every reuse of this operation's inputs: no bottom barrier
@@ -802,13 +821,27 @@ SFC_DEV bool twoshot_op(const KParams& p, int r, int k, int op, uint32_t e, uint
     for (int q = 0; q < N; ++q) src[q] = in_ptr<N>(p, op, q);
     const uint64_t lo = r * sv, hi = min(lo + sv, nvec);
     uint16_t* red = p.red + static_cast<uint64_t>(r) * p.red_stride;
-    for (uint64_t v = lo + gtid; v < hi; v += gstride) {
-      uint4 x[N];
-#pragma unroll
-      for (int q = 0; q < N; ++q) x[q] = load8(src[q], v * 8, count);
+    auto emit = [&](uint64_t v, const uint4(&x)[N]) {
       const uint4 y = reduce8<N>(x);
       *reinterpret_cast<uint4*>(red + (v - lo) * 8) = y;
       store_n(out_r, v * 8, y, 8, count);
+    };
+    constexpr int U = N <= 2 ? 4 : 2;
+    uint64_t v = lo + gtid;
+    for (; v + (U - 1) * gstride < hi; v += U * gstride) {
+      uint4 x[U][N];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int q = 0; q < N; ++q) x[u][q] = load8(src[q], (v + u * gstride) * 8, count);
+#pragma unroll
+      for (int u = 0; u < U; ++u) emit(v + u * gstride, x[u]);
+    }
+    for (; v < hi; v += gstride) {
+      uint4 x[N];
+#pragma unroll
+      for (int q = 0; q < N; ++q) x[q] = load8(src[q], v * 8, count);
+      emit(v, x);
     }
   }
   if (!cta_barrier<N>(p, r, k, op, eb | kPhaseMid)) return false;
@@ -817,10 +850,18 @@ SFC_DEV bool twoshot_op(const KParams& p, int r, int k, int op, uint32_t e, uint
     if (q == r) continue;
     const uint64_t lo = q * sv, hi = min(lo + sv, nvec);
     const uint16_t* red = p.red + static_cast<uint64_t>(q) * p.red_stride;
-    for (uint64_t v = lo + gtid; v < hi; v += gstride) {
-      const uint4 y = ld_rlx_v4u32(red + (v - lo) * 8);
-      store_n(out_r, v * 8, y, 8, count);
+    // eight of the thread's vectors per step (all loads before any store)
+    // while eight remain, then one at a time
+    constexpr int kU = 8;
+    uint64_t v = lo + gtid;
+    for (; v + (kU - 1) * gstride < hi; v += kU * gstride) {
+      uint4 y[kU];
+#pragma unroll
+      for (int i = 0; i < kU; ++i) y[i] = ld_rlx_v4u32(red + (v + i * gstride - lo) * 8);
+#pragma unroll
+      for (int i = 0; i < kU; ++i) store_n(out_r, (v + i * gstride) * 8, y[i], 8, count);
     }
+    for (; v < hi; v += gstride) store_n(out_r, v * 8, ld_rlx_v4u32(red + (v - lo) * 8), 8, count);
   }
   return cta_barrier<N>(p, r, k, op, eb | kPhaseBottom);
 }
