@@ -334,6 +334,7 @@ def run_gpu(args):
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_us, "unit": "us", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h2d,
+                    "min_max": [min(e2e_ms) * 1e3 / K_OPS, max(e2e_ms) * 1e3 / K_OPS],
                     "what": f"sfc_allreduce_chain_host, {K_OPS} ops at {2 * t1['count']} B/rank, per op"},
             "gpu_launches": int(gpu_launches),
             "wall_s": time.perf_counter() - t_start,
