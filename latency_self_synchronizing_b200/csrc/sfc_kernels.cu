@@ -777,7 +777,7 @@ SFC_DEV bool oneshot_op(const KParams& p, int r, int k, int op, uint32_t e, uint
   for (int q = 0; q < N; ++q) src[q] = in_ptr<N>(p, op, q);
   // U of the thread's vectors per step (U * N loads in flight before any
   // use) while U remain, then one at a time
-  constexpr int U = N <= 2 ? 4 : 2;
+  constexpr int U = N <= 2 ? 8 : (N <= 4 ? 4 : 3);
   uint64_t v = gtid;
   for (; v + (U - 1) * gstride < nvec; v += U * gstride) {
     uint4 x[U][N];
@@ -826,7 +826,7 @@ SFC_DEV bool twoshot_op(const KParams& p, int r, int k, int op, uint32_t e, uint
       *reinterpret_cast<uint4*>(red + (v - lo) * 8) = y;
       store_n(out_r, v * 8, y, 8, count);
     };
-    constexpr int U = N <= 2 ? 4 : 2;
+    constexpr int U = N <= 2 ? 8 : (N <= 4 ? 4 : 3);
     uint64_t v = lo + gtid;
     for (; v + (U - 1) * gstride < hi; v += U * gstride) {
       uint4 x[U][N];
