@@ -299,6 +299,36 @@ def run_gpu(args):
     e2e_us = statistics.median(e2e_ms) * 1e3 / K_OPS
     h2d = hin.numel() * 2
 
+    # single calls (one launch per all-reduce, launch included): reported
+    # beside the chained latency, not the headline
+    xs = [torch.from_numpy(t1["x"][0, r].view(np.int16)).view(torch.bfloat16).to(dev) for r in range(NRANKS)]
+    ys = [torch.empty_like(t) for t in xs]
+    for _ in range(20):
+        comm.allreduce(xs, ys, protocol=PROTOCOL)
+    torch.cuda.synchronize()
+    n_calls = 200
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n_calls):
+        comm.allreduce(xs, ys, protocol=PROTOCOL)
+    b.record(stream)
+    torch.cuda.synchronize()
+    single_b2b = a.elapsed_time(b) * 1e3 / n_calls
+    iso = []
+    for _ in range(50):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        comm.allreduce(xs, ys, protocol=PROTOCOL)
+        b.record(stream)
+        torch.cuda.synchronize()
+        iso.append(a.elapsed_time(b) * 1e3)
+    single = {"back_to_back_us": single_b2b, "isolated_us_p50": _percentile(iso, 0.5), "unit": "us",
+              "what": f"sfc_allreduce, one launch per call, {2 * t1['count']} B/rank; back to back = "
+                      f"{n_calls} calls between two events; isolated = one call between two events"}
+    st, info = comm.status()
+    if st != api.Status.OK:
+        raise RuntimeError(f"device status {st.name} info {info:#x}")
+
     head = per_size[0]
     value = head["p50_us"]
     value, e2e_us = reduce_max_over_ranks([value, e2e_us], device=dev)
@@ -336,6 +366,7 @@ def run_gpu(args):
             "e2e": {"value": e2e_us, "unit": "us", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h2d,
                     "min_max": [min(e2e_ms) * 1e3 / K_OPS, max(e2e_ms) * 1e3 / K_OPS],
                     "what": f"sfc_allreduce_chain_host, {K_OPS} ops at {2 * t1['count']} B/rank, per op"},
+            "single_call": single,
             "gpu_launches": int(gpu_launches),
             "wall_s": time.perf_counter() - t_start,
             "clocks": clk,

@@ -35,8 +35,9 @@
  *     after the call's kernel has finished and never writes an input.
  *   - Epochs: 32-bit, start at 1 after sfc_init / sfc_reset; every
  *     operation consumes one, and a call must pass exactly the next one
- *     (sfc_next_epoch), else SFC_ERR_EPOCH. All-reduce and all-gather share
- *     the sequence. Parity = epoch & 1 selects the scratch buffer.
+ *     (sfc_next_epoch), else SFC_ERR_EPOCH; 0, never an epoch itself,
+ *     stands for the next one. All-reduce and all-gather share the
+ *     sequence. Parity = epoch & 1 selects the scratch buffer.
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*,
  *     NULL = the legacy default stream). Calls on one context must be
  *     ordered on the GPU (one stream, or streams joined by events).

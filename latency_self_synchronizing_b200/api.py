@@ -84,9 +84,16 @@ def _check(rc, what):
         raise SfcError(rc, what)
 
 
-def _stream_handle(stream):
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return C.c_void_p(s.cuda_stream)
+_raw_current_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream_handle(stream, device=None):
+    """cudaStream_t of `stream`, or of the device's current stream."""
+    if stream is not None:
+        return C.c_void_p(stream.cuda_stream)
+    if _raw_current_stream is not None and device is not None:
+        return C.c_void_p(_raw_current_stream(device))
+    return C.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
 def _dev_ptr(t, name):
@@ -125,6 +132,9 @@ class Communicator:
         self._ctx = handle
         self.nranks = int(nranks)
         self.max_bytes_per_rank = int(max_bytes_per_rank)
+        self._device = torch.cuda.current_device()
+        self._ptrs_in = (C.c_void_p * self.nranks)()
+        self._ptrs_out = (C.c_void_p * self.nranks)()
 
     # ----------------------------------------------------------- lifecycle
     def close(self):
@@ -167,22 +177,34 @@ class Communicator:
 
     # --------------------------------------------------------- collectives
     def _one(self, fn, op, inputs, outputs, protocol, epoch, stream):
+        # per-call cost matters here (one launch per all-reduce): checks are
+        # plain attribute reads, the pointer arrays are reused, the epoch is
+        # left to the library (0 = next) and the stream read without a
+        # Stream object
         n = self.nranks
         if len(inputs) != n or len(outputs) != n:
             raise ValueError(f"need {n} inputs and {n} outputs")
         count = inputs[0].numel()
-        for t in inputs:
-            if t.numel() != count:
-                raise ValueError("all inputs must have the same number of elements")
         want_out = count if op == Op.ALLREDUCE else n * count
-        for t in outputs:
-            if t.numel() != want_out:
+        ins, outs = self._ptrs_in, self._ptrs_out
+        bf16 = torch.bfloat16
+        for r in range(n):
+            a, b = inputs[r], outputs[r]
+            if not (a.is_cuda and b.is_cuda and a.dtype is bf16 and b.dtype is bf16 and a.is_contiguous()
+                    and b.is_contiguous()):
+                _dev_ptr(a, "input")
+                _dev_ptr(b, "output")
+            if a.numel() != count:
+                raise ValueError("all inputs must have the same number of elements")
+            if b.numel() != want_out:
                 raise ValueError(f"outputs must have {want_out} elements")
-        ins = (C.c_void_p * n)(*[_dev_ptr(t, "input") for t in inputs])
-        outs = (C.c_void_p * n)(*[_dev_ptr(t, "output") for t in outputs])
-        e = self.next_epoch if epoch is None else int(epoch)
-        _check(fn(self._ctx, ins, outs, count, 0, int(as_protocol(protocol)), e, _stream_handle(stream)),
-               fn.__name__)
+            ins[r] = a.data_ptr()
+            outs[r] = b.data_ptr()
+        proto = protocol if type(protocol) is int else int(as_protocol(protocol))
+        e = 0 if epoch is None else int(epoch)
+        rc = fn(self._ctx, ins, outs, count, 0, proto, e, _stream_handle(stream, self._device))
+        if rc != 0:
+            raise SfcError(rc, fn.__name__)
 
     def allreduce(self, inputs, outputs, protocol="auto", epoch=None, stream=None):
         """outputs[r] = rank-order fp32 sum of inputs, rounded once to bf16."""

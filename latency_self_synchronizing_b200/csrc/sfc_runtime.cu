@@ -195,9 +195,13 @@ sfc_status prepare_timings(uint64_t* timings, int k_ops, cudaStream_t stream) {
   return SFC_OK;
 }
 
+// Epoch 0 is never a valid epoch; callers pass it for "the next one".
+uint32_t resolve_epoch(const sfc_ctx* c, uint32_t e) { return e == 0 ? c->next_epoch : e; }
+
 sfc_status one_op(sfc_ctx* c, sfc_op op, const void* const* in, void* const* out, size_t count, sfc_dtype dtype,
                   sfc_protocol protocol, uint32_t epoch, void* stream) {
   if (c == nullptr || in == nullptr || out == nullptr) return SFC_ERR_INVALID;
+  epoch = resolve_epoch(c, epoch);
   if (count == 0) return (dtype == SFC_BF16) ? SFC_OK : SFC_ERR_UNSUPPORTED;
   int proto = protocol;
   if (proto == SFC_PROTO_AUTO) proto = sfc_select_protocol(c, op, count * 2, c->nranks);
@@ -232,6 +236,7 @@ sfc_status chain(sfc_ctx* c, sfc_op op, int k_ops, const void* const* in_table, 
                  sfc_dtype dtype, sfc_protocol protocol, uint32_t first_epoch, const uint32_t* skew_ns,
                  uint64_t* timings, void* stream) {
   if (c == nullptr || in_table == nullptr || out_table == nullptr) return SFC_ERR_INVALID;
+  first_epoch = resolve_epoch(c, first_epoch);
   if (count == 0) return (dtype == SFC_BF16 && k_ops >= 1) ? SFC_OK : SFC_ERR_INVALID;
   int proto = protocol;
   if (proto == SFC_PROTO_AUTO) proto = sfc_select_protocol(c, op, count * 2, c->nranks);
@@ -537,6 +542,7 @@ sfc_status sfc_allreduce_chain_host(sfc_ctx* c, int k_ops, const void* in_host, 
                                     sfc_dtype dtype, sfc_protocol protocol, uint32_t first_epoch, uint64_t* timings,
                                     void* stream) {
   if (c == nullptr || in_host == nullptr || out_host == nullptr || k_ops < 1) return SFC_ERR_INVALID;
+  first_epoch = resolve_epoch(c, first_epoch);
   if (count == 0) return dtype == SFC_BF16 ? SFC_OK : SFC_ERR_UNSUPPORTED;
   int proto = protocol;
   if (proto == SFC_PROTO_AUTO) proto = sfc_select_protocol(c, SFC_OP_ALLREDUCE, count * 2, c->nranks);
@@ -709,6 +715,7 @@ sfc_status sfc_linear_allreduce(sfc_ctx* c, const void* const* W, const void* co
     return SFC_ERR_INVALID;
   if (c->region[kLL] == nullptr) return SFC_ERR_UNSUPPORTED;
   if (c->poisoned) return SFC_ERR_ABORTED;
+  epoch = resolve_epoch(c, epoch);
   if (epoch != c->next_epoch) return SFC_ERR_EPOCH;
   const int N = c->nranks;
   sfc::LinearParams p{};
