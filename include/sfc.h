@@ -151,7 +151,11 @@ typedef struct {
  * (all-gather: per shard). Allocates the scratch (per provisioned protocol:
  * 2 parities x N x (N-1) encoded slots), barrier flags and status words;
  * sentinel slots are filled with 0xFFFF, flags zeroed, next epoch = 1.
- * cfg may be NULL (defaults). Synchronous. */
+ * cfg may be NULL (defaults). Synchronous. Environment, read here:
+ * SFC_TIMEOUT_MS (> 0) bounds every device wait when cfg leaves timeout_us
+ * at 0; SFC_PROTOCOL (a protocol name such as "sentinel", lower case, or its
+ * number) is what AUTO resolves to wherever that protocol is provisioned
+ * and supports the operation. Unparsable values are ignored. */
 sfc_status sfc_init(sfc_ctx** ctx, int nranks, size_t max_bytes_per_rank, const sfc_config* cfg);
 
 /* Free everything the context owns (synchronizes the device first). */

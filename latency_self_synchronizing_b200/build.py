@@ -1,11 +1,16 @@
 """Build libsfc.so in-tree with nvcc for sm_100a.
 
-    python -m latency_self_synchronizing_b200.build [--force] [--verbose]
+    python -m latency_self_synchronizing_b200.build [--force] [--verbose] [--debug]
 
 Compiles every .cu under csrc/ to an object (in parallel, skipping objects
 newer than their sources and headers) and links them into
 latency_self_synchronizing_b200/libsfc.so against the static CUDA runtime.
 No fast-math: fp32 adds must round to nearest with subnormals kept.
+
+--debug builds libsfc_debug.so instead (objects in _build_debug/) with
+-DSFC_DEBUG: every scratch access is checked against its protocol region and
+one outside it is recorded as SFC_ERR_GUARD and skipped. Select it at run
+time with SFC_LIB=<path to libsfc_debug.so>.
 """
 
 import argparse
@@ -21,6 +26,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libsfc.so")
+BUILD_DEBUG = os.path.join(PKG, "_build_debug")
+LIB_DEBUG = os.path.join(PKG, "libsfc_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-I", INCLUDE, "-I", CSRC]
@@ -50,18 +57,21 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force=False, verbose=False, ptxas_verbose=False):
-    """Compile and link; returns the path of libsfc.so."""
+def build(force=False, verbose=False, ptxas_verbose=False, debug=False):
+    """Compile and link; returns the path of libsfc.so (libsfc_debug.so with
+    debug=True)."""
     nvcc = _nvcc()
-    os.makedirs(BUILD, exist_ok=True)
+    bdir, lib = (BUILD_DEBUG, LIB_DEBUG) if debug else (BUILD, LIB)
+    flags = FLAGS + (["-DSFC_DEBUG"] if debug else [])
+    os.makedirs(bdir, exist_ok=True)
     headers = _headers()
     jobs = []
     objs = []
     for src in _sources():
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(bdir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if force or _stale(obj, [src] + headers):
-            cmd = [nvcc] + ARCH + FLAGS + (["-Xptxas", "-v"] if ptxas_verbose else []) + ["-c", src, "-o", obj]
+            cmd = [nvcc] + ARCH + flags + (["-Xptxas", "-v"] if ptxas_verbose else []) + ["-c", src, "-o", obj]
             jobs.append(cmd)
 
     def run(cmd):
@@ -76,10 +86,10 @@ def build(force=False, verbose=False, ptxas_verbose=False):
 
     with cf.ThreadPoolExecutor(max_workers=max(1, min(len(jobs), os.cpu_count() or 1))) as ex:
         list(ex.map(run, jobs))
-    if force or jobs or _stale(LIB, objs):
-        link = [nvcc] + ARCH + ["-shared", "-cudart", "static", "-o", LIB] + objs
+    if force or jobs or _stale(lib, objs):
+        link = [nvcc] + ARCH + ["-shared", "-cudart", "static", "-o", lib] + objs
         run(link)
-    return LIB
+    return lib
 
 
 def main(argv=None):
@@ -87,8 +97,9 @@ def main(argv=None):
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas", action="store_true", help="print register / spill statistics")
+    ap.add_argument("--debug", action="store_true", help="build libsfc_debug.so with scratch bounds checks")
     a = ap.parse_args(argv)
-    print(build(force=a.force, verbose=a.verbose, ptxas_verbose=a.ptxas))
+    print(build(force=a.force, verbose=a.verbose, ptxas_verbose=a.ptxas, debug=a.debug))
 
 
 if __name__ == "__main__":

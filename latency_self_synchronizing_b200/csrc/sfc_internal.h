@@ -83,6 +83,7 @@ struct KParams {
                         // the twoshot protocols keep their all-gather slots
                         // after the 2 * N * (N - 1) reduce-scatter slots
   uint64_t slot_stride; // bytes
+  uint64_t scratch_bytes;  // size of the protocol region (debug builds check every access)
   uint64_t* bar;        // barrier counters [N][bar_stride]
   int bar_stride;
   uint16_t* red;        // twoshot reduced shards [N][red_stride]

@@ -80,6 +80,31 @@ struct Operands {
   const uint16_t* in_next;  // null on the last operation
 };
 
+// Scratch access check. A build with -DSFC_DEBUG tests every scratch access
+// against the protocol's region; one out of it records SFC_ERR_GUARD (detail =
+// the offset from the region start) and is skipped, so the waits then end on
+// the abort word instead of the access touching memory outside the region.
+// Normal builds compile the check away.
+SFC_DEV bool scratch_in_bounds(const KParams& p, const void* ptr, uint64_t bytes) {
+  const uint8_t* a = static_cast<const uint8_t*>(ptr);
+  if (a >= p.scratch && a + bytes <= p.scratch + p.scratch_bytes) return true;
+  record_error(p, 9 /* SFC_ERR_GUARD */, static_cast<uint32_t>(a - p.scratch));
+  return false;
+}
+#ifdef SFC_DEBUG
+#define SFC_SCRATCH(p, ptr, bytes, ...)            \
+  do {                                              \
+    if (scratch_in_bounds(p, ptr, bytes)) {         \
+      __VA_ARGS__;                                  \
+    }                                               \
+  } while (0)
+#else
+#define SFC_SCRATCH(p, ptr, bytes, ...) \
+  do {                                  \
+    __VA_ARGS__;                        \
+  } while (0)
+#endif
+
 // LL layout shared with the public device API (one definition).
 SFC_DEV uint64_t ll_off(uint64_t v, int half) { return sfc_device::ll_offset(v, half); }
 
@@ -119,8 +144,8 @@ SFC_DEV bool ll_poll(const KParams& p, int r, int op, uint32_t e, uint64_t gtid,
         for (int j = 0; j < N - 1; ++j) {
           if (cur & (1u << (i * (N - 1) + j))) {
             const uint8_t* s = my + static_cast<uint64_t>(j) * p.slot_stride;
-            ld_rlx_v2u64(s + o0, a[i][j], b[i][j]);
-            ld_rlx_v2u64(s + o1, c[i][j], d[i][j]);
+            SFC_SCRATCH(p, s + o0, 16, ld_rlx_v2u64(s + o0, a[i][j], b[i][j]));
+            SFC_SCRATCH(p, s + o1, 16, ld_rlx_v2u64(s + o1, c[i][j], d[i][j]));
           }
         }
       }
@@ -184,8 +209,8 @@ SFC_DEV bool ll_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid, u
       for (int q = 0; q < N; ++q) {
         if (q == r) continue;
         uint8_t* s = slot_ptr<N>(p, q, par, r);
-        st_rlx_v2u64(s + o0, ehi | x.x, ehi | x.y);
-        st_rlx_v2u64(s + o1, ehi | x.z, ehi | x.w);
+        SFC_SCRATCH(p, s + o0, 16, st_rlx_v2u64(s + o0, ehi | x.x, ehi | x.y));
+        SFC_SCRATCH(p, s + o1, 16, st_rlx_v2u64(s + o1, ehi | x.z, ehi | x.w));
       }
     }
   }
@@ -228,8 +253,8 @@ SFC_DEV bool sentinel_poll(const KParams& p, int r, int op, uint64_t gtid, uint6
         for (int j = 0; j < N - 1; ++j) {
           const int u = 2 * (i * (N - 1) + j);
           uint8_t* s = my + static_cast<uint64_t>(j) * p.slot_stride + v[i] * 16;
-          if (cur & (1u << u)) a[i][j] = atom_exch_u64(s, kFill);
-          if (cur & (2u << u)) b[i][j] = atom_exch_u64(s + 8, kFill);
+          if (cur & (1u << u)) SFC_SCRATCH(p, s, 8, a[i][j] = atom_exch_u64(s, kFill));
+          if (cur & (2u << u)) SFC_SCRATCH(p, s + 8, 8, b[i][j] = atom_exch_u64(s + 8, kFill));
         }
       }
 #pragma unroll
@@ -296,7 +321,8 @@ SFC_DEV bool sentinel_op(const KParams& p, int r, int op, uint32_t e, uint64_t g
 #pragma unroll
       for (int q = 0; q < N; ++q) {
         if (q == r) continue;
-        st_rlx_v2u64(slot_ptr<N>(p, q, par, r) + v * 16, lo, hi);
+        uint8_t* s = slot_ptr<N>(p, q, par, r) + v * 16;
+        SFC_SCRATCH(p, s, 16, st_rlx_v2u64(s, lo, hi));
       }
     }
   }
@@ -348,9 +374,9 @@ SFC_DEV bool ll128_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid
           if (q == r) continue;
           uint8_t* s = slot_ptr<N>(p, q, par, r) + L * kLL128Line + sub * 16;
           if (sub < 7)
-            st_rlx_v4u32(s, make_uint4(lo.x, lo.y, hi.x, hi.y));
+            SFC_SCRATCH(p, s, 16, st_rlx_v4u32(s, make_uint4(lo.x, lo.y, hi.x, hi.y)));
           else
-            st_rlx_v2u32(s, lo);
+            SFC_SCRATCH(p, s, 8, st_rlx_v2u32(s, lo));
         }
       }
     }
@@ -362,7 +388,8 @@ SFC_DEV bool ll128_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid
 #pragma unroll
         for (int q = 0; q < N; ++q) {
           if (q == r) continue;
-          st_rlx_u64(slot_ptr<N>(p, q, par, r) + L * kLL128Line + 120, static_cast<uint64_t>(e));
+          uint8_t* fl = slot_ptr<N>(p, q, par, r) + L * kLL128Line + 120;
+          SFC_SCRATCH(p, fl, 8, st_rlx_u64(fl, static_cast<uint64_t>(e)));
         }
       }
     }
@@ -400,7 +427,8 @@ SFC_DEV bool ll128_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid
         for (int q = 0; q < N; ++q) {
           if (cur & (1u << (b * N + q))) {
             const int j = q < r ? q : q - 1;
-            f[b * N + q] = ld_rlx_u64(my + static_cast<uint64_t>(j) * p.slot_stride + L * kLL128Line + 120);
+            const uint8_t* fl = my + static_cast<uint64_t>(j) * p.slot_stride + L * kLL128Line + 120;
+            SFC_SCRATCH(p, fl, 8, f[b * N + q] = ld_rlx_u64(fl));
           }
         }
       }
@@ -431,9 +459,10 @@ SFC_DEV bool ll128_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid
           const int j = q < r ? q : q - 1;
           const uint8_t* s = my + static_cast<uint64_t>(j) * p.slot_stride + L * kLL128Line + sub * 16;
           if (sub < 7) {
-            x[q] = ld_rlx_v4u32(s);
+            SFC_SCRATCH(p, s, 16, x[q] = ld_rlx_v4u32(s));
           } else {
-            const uint2 t = ld_rlx_v2u32(s);
+            uint2 t = make_uint2(0, 0);
+            SFC_SCRATCH(p, s, 8, t = ld_rlx_v2u32(s));
             x[q] = make_uint4(t.x, t.y, 0u, 0u);
           }
         }
@@ -468,12 +497,16 @@ struct TwoshotSlots {
 
 // Store one 8-element vector into a slot position v, encoded.
 template <bool kLLenc>
-SFC_DEV void push_vec(uint8_t* slot, uint64_t v, uint4 x, uint64_t ehi) {
+SFC_DEV void push_vec(const KParams& p, uint8_t* slot, uint64_t v, uint4 x, uint64_t ehi) {
   if (kLLenc) {
-    st_rlx_v2u64(slot + ll_off(v, 0), ehi | x.x, ehi | x.y);
-    st_rlx_v2u64(slot + ll_off(v, 1), ehi | x.z, ehi | x.w);
+    uint8_t* s0 = slot + ll_off(v, 0);
+    uint8_t* s1 = slot + ll_off(v, 1);
+    SFC_SCRATCH(p, s0, 16, st_rlx_v2u64(s0, ehi | x.x, ehi | x.y));
+    SFC_SCRATCH(p, s1, 16, st_rlx_v2u64(s1, ehi | x.z, ehi | x.w));
   } else {
-    st_rlx_v2u64(slot + v * 16, (static_cast<uint64_t>(x.y) << 32) | x.x, (static_cast<uint64_t>(x.w) << 32) | x.z);
+    uint8_t* s = slot + v * 16;
+    SFC_SCRATCH(p, s, 16,
+                st_rlx_v2u64(s, (static_cast<uint64_t>(x.y) << 32) | x.x, (static_cast<uint64_t>(x.w) << 32) | x.z));
   }
 }
 
@@ -502,12 +535,12 @@ SFC_DEV bool poll_vecs(const KParams& p, uint8_t* base, uint64_t v, uint32_t e, 
       uint8_t* sq = base + static_cast<uint64_t>(q < r ? q : q - 1) * p.slot_stride;
       if (kLLenc) {
         if (cur & (1u << q)) {
-          ld_rlx_v2u64(sq + ll_off(v, 0), a[q], b[q]);
-          ld_rlx_v2u64(sq + ll_off(v, 1), c[q], d[q]);
+          SFC_SCRATCH(p, sq + ll_off(v, 0), 16, ld_rlx_v2u64(sq + ll_off(v, 0), a[q], b[q]));
+          SFC_SCRATCH(p, sq + ll_off(v, 1), 16, ld_rlx_v2u64(sq + ll_off(v, 1), c[q], d[q]));
         }
       } else {
-        if (cur & (1u << (2 * q))) a[q] = atom_exch_u64(sq + v * 16, kFill);
-        if (cur & (2u << (2 * q))) b[q] = atom_exch_u64(sq + v * 16 + 8, kFill);
+        if (cur & (1u << (2 * q))) SFC_SCRATCH(p, sq + v * 16, 8, a[q] = atom_exch_u64(sq + v * 16, kFill));
+        if (cur & (2u << (2 * q))) SFC_SCRATCH(p, sq + v * 16 + 8, 8, b[q] = atom_exch_u64(sq + v * 16 + 8, kFill));
       }
     }
 #pragma unroll
@@ -558,7 +591,7 @@ SFC_DEV bool selfsync_twoshot_op(const KParams& p, int r, int op, uint32_t e, ui
       for (int s = 0; s < N; ++s) {
         if (s == r) continue;
         const uint64_t vg = s * sv + v;
-        if (vg < nvec) push_vec<kLLenc>(S::rs(p, s, par, r), v, load8(in_r, vg * 8, count), ehi);
+        if (vg < nvec) push_vec<kLLenc>(p, S::rs(p, s, par, r), v, load8(in_r, vg * 8, count), ehi);
       }
     }
   }
@@ -595,7 +628,7 @@ SFC_DEV bool selfsync_twoshot_op(const KParams& p, int r, int op, uint32_t e, ui
         if (r != p.silent_rank) {
 #pragma unroll
           for (int q = 0; q < N; ++q)
-            if (q != r) push_vec<kLLenc>(S::ag(p, q, par, r), v, y, ehi);
+            if (q != r) push_vec<kLLenc>(p, S::ag(p, q, par, r), v, y, ehi);
         }
       }
     }
@@ -661,7 +694,8 @@ SFC_DEV bool ll128_fast_op(const KParams& p, int r, int op, uint32_t e, uint64_t
 #pragma unroll
         for (int q = 0; q < N; ++q) {
           if (q == r) continue;
-          st_rlx_v2u64(slot_ptr<N>(p, q, par, r) + L * kLL128Line + sub * 16, a, b);
+          uint8_t* s = slot_ptr<N>(p, q, par, r) + L * kLL128Line + sub * 16;
+          SFC_SCRATCH(p, s, 16, st_rlx_v2u64(s, a, b));
         }
       }
     }
@@ -686,8 +720,10 @@ SFC_DEV bool ll128_fast_op(const KParams& p, int r, int op, uint32_t e, uint64_t
       const uint32_t cur = need;
 #pragma unroll
       for (int j = 0; j < N - 1; ++j)
-        if (cur & (1u << j))
-          ld_rlx_v2u64(my + static_cast<uint64_t>(j) * p.slot_stride + L * kLL128Line + sub * 16, a[j], b[j]);
+        if (cur & (1u << j)) {
+          const uint8_t* s = my + static_cast<uint64_t>(j) * p.slot_stride + L * kLL128Line + sub * 16;
+          SFC_SCRATCH(p, s, 16, ld_rlx_v2u64(s, a[j], b[j]));
+        }
       // the flag lane decides for its line; the other 7 lanes take its verdict
       uint32_t okbits = 0;
 #pragma unroll

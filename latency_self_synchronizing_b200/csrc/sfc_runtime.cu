@@ -42,6 +42,7 @@ struct sfc_ctx {
   sfc_cost_model model{};
 
   int occupancy[kNumProtocols][2][2] = {};  // blocks per SM, per (protocol, op, CTA size), 0 = unknown
+  int forced_protocol = 0;                // SFC_PROTOCOL: what AUTO resolves to (0 = the selector)
   int smem_optin = 0;                     // opt-in shared memory per block (bytes)
   int linear_occ = 0;                     // fused-linear CTAs per SM (0 = not yet queried)
 
@@ -159,6 +160,7 @@ void fill_common(sfc_ctx* c, KParams& p, int proto, uint64_t count, int k_ops, u
   p.first_epoch = first_epoch;
   p.scratch = self_sync(proto) ? c->region[proto] : nullptr;
   p.slot_stride = self_sync(proto) ? c->slot_stride[proto] : 0;
+  p.scratch_bytes = self_sync(proto) ? c->region_bytes[proto] : 0;
   p.bar = c->bar;
   p.bar_stride = c->bar_stride;
   p.red = c->red;
@@ -257,6 +259,35 @@ sfc_status chain(sfc_ctx* c, sfc_op op, int k_ops, const void* const* in_table, 
   s = launch(c, proto, op, p, st);
   if (s == SFC_OK) c->next_epoch = first_epoch + static_cast<uint32_t>(k_ops);
   return s;
+}
+
+// Environment overrides, read once per context:
+//   SFC_TIMEOUT_MS  bound on every device wait (ms, > 0), used when the
+//                   config leaves timeout_us at 0;
+//   SFC_PROTOCOL    the protocol AUTO resolves to (a name as in the Python
+//                   binding, e.g. "sentinel", or its number), wherever that
+//                   protocol is provisioned and supports the operation.
+// Unparsable values are ignored.
+void apply_env_overrides(sfc_ctx* c) {
+  if (const char* t = std::getenv("SFC_TIMEOUT_MS")) {
+    char* end = nullptr;
+    const long ms = std::strtol(t, &end, 10);
+    if (end != t && *end == '\0' && ms > 0 && ms <= 4000000 && c->cfg.timeout_us == 0)
+      c->cfg.timeout_us = static_cast<uint32_t>(ms * 1000);
+  }
+  if (const char* pstr = std::getenv("SFC_PROTOCOL")) {
+    static const char* const names[kNumProtocols] = {"auto",       "ll",          "ll128",
+                                                     "sentinel",   "barrier_oneshot", "barrier_twoshot",
+                                                     "barrier_oneshot_db", "ll_twoshot", "sentinel_twoshot",
+                                                     "ll128_fast"};
+    int f = 0;
+    for (int i = 1; i < kNumProtocols; ++i)
+      if (std::strcmp(pstr, names[i]) == 0) f = i;
+    char* end = nullptr;
+    const long v = std::strtol(pstr, &end, 10);
+    if (f == 0 && end != pstr && *end == '\0' && v > 0 && v < kNumProtocols) f = static_cast<int>(v);
+    c->forced_protocol = f;
+  }
 }
 
 // Built-in latency model: the p50 latencies the message-size sweep measured
@@ -403,6 +434,8 @@ sfc_protocol sfc_select_protocol_model(const sfc_cost_model* m, sfc_op op, size_
 
 sfc_protocol sfc_select_protocol(const sfc_ctx* c, sfc_op op, size_t bytes_per_rank, int nranks) {
   if (c == nullptr) return SFC_PROTO_AUTO;
+  const int f = c->forced_protocol;
+  if (f != 0 && provisioned(c, f) && !(op == SFC_OP_ALLGATHER && twoshot_alg(f))) return static_cast<sfc_protocol>(f);
   sfc_cost_model m = c->model;
   // protocols without scratch in this context are never chosen
   for (int pr = 1; pr < SFC_NUM_PROTOCOLS; ++pr)
@@ -426,6 +459,7 @@ sfc_status sfc_init(sfc_ctx** out, int nranks, size_t max_bytes_per_rank, const 
   if (cfg && (cfg->protocol_mask & ~kAllProtocolsMask)) return SFC_ERR_INVALID;
   sfc_ctx* c = new sfc_ctx();
   if (cfg) c->cfg = *cfg;
+  apply_env_overrides(c);
   c->nranks = nranks;
   c->max_bytes = max_bytes_per_rank;
   c->max_count = max_bytes_per_rank / 2;

@@ -31,6 +31,17 @@ def test_library_exports_every_declared_symbol():
     assert set(names) == {s[0] for s in _lib.SIGNATURES}
 
 
+def test_debug_library_exports_the_same_symbols():
+    """The bounds-checked build (built by __graft_entry__.build) is the same ABI."""
+    import ctypes
+    path = os.path.join(os.path.dirname(_lib.LIB_PATH), "libsfc_debug.so")
+    if not os.path.exists(path):
+        pytest.skip("libsfc_debug.so not built")
+    lib = ctypes.CDLL(path)
+    for n in _declared():
+        assert hasattr(lib, n), n
+
+
 def test_status_strings():
     for s in api.Status:
         assert api.status_string(s)

@@ -106,3 +106,64 @@ def test_zero_count_is_a_noop():
         assert comm.next_epoch == e and comm.launch_count == 0
     finally:
         comm.close()
+
+
+def test_epoch_zero_means_next():
+    """0 is never an epoch; every entry point reads it as the next one."""
+    import ctypes as C
+    comm = api.Communicator(2, 4096)
+    try:
+        x = make_inputs(seed=5, k_ops=3, nranks=2, count=64)
+        ins, outs = _ops(x)
+        lib = comm._lib
+        for k in range(3):
+            pi = (C.c_void_p * 2)(*[t.data_ptr() for t in ins.tensors(k)])
+            po = (C.c_void_p * 2)(*[t.data_ptr() for t in outs.tensors(k)])
+            assert lib.sfc_allreduce(comm._ctx, pi, po, 64, 0, int(api.Protocol.LL), 0, None) == 0
+            assert comm.next_epoch == 2 + k
+        torch.cuda.synchronize()
+        assert comm.status()[0] == api.Status.OK
+        for k in range(3):
+            np.testing.assert_array_equal(outs.bits()[k, 0], reference.allreduce(x[k]))
+        with pytest.raises(api.SfcError) as ei:  # an explicit stale epoch is still refused
+            comm.allreduce(ins.tensors(0), outs.tensors(0), protocol="ll", epoch=1)
+        assert ei.value.status == api.Status.EPOCH
+    finally:
+        comm.close()
+
+
+def test_env_overrides(monkeypatch):
+    """SFC_PROTOCOL forces what AUTO resolves to; SFC_TIMEOUT_MS bounds the
+    device waits (a silent rank times out within it)."""
+    import time
+    monkeypatch.setenv("SFC_PROTOCOL", "barrier_oneshot_db")
+    monkeypatch.setenv("SFC_TIMEOUT_MS", "3")
+    comm = api.Communicator(4, 1 << 14)
+    try:
+        assert comm.select_protocol("allreduce", 2048) == api.Protocol.BARRIER_ONESHOT_DB
+        assert comm.select_protocol("allgather", 2048) == api.Protocol.BARRIER_ONESHOT_DB
+        x = make_inputs(seed=6, k_ops=2, nranks=4, count=1024)
+        ins, outs = _ops(x)
+        comm.allreduce_chain(ins.table, outs.table, 1024, 2, protocol="auto")
+        torch.cuda.synchronize()
+        assert comm.status()[0] == api.Status.OK
+        for k in range(2):
+            np.testing.assert_array_equal(outs.bits()[k, 1], reference.allreduce(x[k]))
+        comm.set_silent_rank(1)
+        t0 = time.perf_counter()
+        comm.allreduce_chain(ins.table, outs.table, 1024, 2, protocol="ll")
+        torch.cuda.synchronize()
+        assert time.perf_counter() - t0 < 1.0
+        assert comm.status()[0] == api.Status.TIMEOUT
+        comm.set_silent_rank(-1)
+        comm.reset()
+    finally:
+        comm.close()
+    monkeypatch.setenv("SFC_PROTOCOL", "ll_twoshot")  # all-reduce only: all-gather keeps the selector
+    monkeypatch.setenv("SFC_TIMEOUT_MS", "not a number")
+    comm = api.Communicator(4, 1 << 14)
+    try:
+        assert comm.select_protocol("allreduce", 2048) == api.Protocol.LL_TWOSHOT
+        assert comm.select_protocol("allgather", 2048) != api.Protocol.LL_TWOSHOT
+    finally:
+        comm.close()
