@@ -274,6 +274,7 @@ def run_gpu(args):
             "mean_us_from_events": mean_launch_us / K_OPS,
             "algorithmic_bytes_per_op": bytes_op,
             "achieved_gbs_p50": bytes_op / (p50 * 1e-6) / 1e9 if p50 > 0 else None,
+            "algbw_gbs_p50": 2 * count / (p50 * 1e-6) / 1e9 if p50 > 0 else None,
             "achieved_gbs_launch": bytes_op * K_OPS / (mean_launch_us * 1e-6) / 1e9,
             "floor_ratio_p50": p50 / (floor["flag_rtt_ns_p50"] / 1e3),
             "launch_shape": comm.launch_shape("allreduce", PROTOCOL, count),

@@ -75,6 +75,7 @@ def measure_point(comm, op, proto, count, k_ops, reps, gen, dev):
     return {"op": op, "protocol": proto, "nranks": n, "bytes_per_rank": 2 * count, "count": count,
             "p50_us": p50, "p99_us": _percentile(lat, 0.99), "mean_us_events": statistics.mean(ev_us),
             "algorithmic_bytes": nbytes, "gbs_p50": nbytes / (p50 * 1e-6) / 1e9 if p50 > 0 else None,
+            "algbw_gbs_p50": 2 * count / (p50 * 1e-6) / 1e9 if p50 > 0 else None,
             "ctas_per_rank": comm.launch_shape(op, proto, count)[0]}
 
 
