@@ -323,9 +323,39 @@ def run_gpu(args):
         b.record(stream)
         torch.cuda.synchronize()
         iso.append(a.elapsed_time(b) * 1e3)
-    single = {"back_to_back_us": single_b2b, "isolated_us_p50": _percentile(iso, 0.5), "unit": "us",
+    # the same calls captured in a CUDA graph (device-epoch context) and
+    # replayed: launch gaps on the GPU only, no host work per call
+    gcomm = api.Communicator(NRANKS, 2 * t1["count"], device_epochs=True, protocols=[PROTOCOL])
+    gys = [torch.empty_like(t) for t in xs]
+    gcomm.allreduce(xs, gys, protocol=PROTOCOL)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(K_OPS):
+            gcomm.allreduce(xs, gys, protocol=PROTOCOL)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    g_us = []
+    for _ in range(5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        graph.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        g_us.append(a.elapsed_time(b) * 1e3 / K_OPS)
+    gst, ginfo = gcomm.status()
+    if gst != api.Status.OK:
+        raise RuntimeError(f"graph context status {gst.name} info {ginfo:#x}")
+    if not torch.equal(gys[0], ys[0]):
+        raise RuntimeError("graph-replayed all-reduce differs from the eager one")
+    del graph
+    gcomm.close()
+    single = {"back_to_back_us": single_b2b, "isolated_us_p50": _percentile(iso, 0.5),
+              "graph_replay_us": statistics.median(g_us), "unit": "us",
               "what": f"sfc_allreduce, one launch per call, {2 * t1['count']} B/rank; back to back = "
-                      f"{n_calls} calls between two events; isolated = one call between two events"}
+                      f"{n_calls} calls between two events; isolated = one call between two events; "
+                      f"graph replay = {K_OPS} calls captured in one CUDA graph (device epochs), per call"}
     st, info = comm.status()
     if st != api.Status.OK:
         raise RuntimeError(f"device status {st.name} info {info:#x}")

@@ -38,6 +38,15 @@
  *     (sfc_next_epoch), else SFC_ERR_EPOCH; 0, never an epoch itself,
  *     stands for the next one. All-reduce and all-gather share the
  *     sequence. Parity = epoch & 1 selects the scratch buffer.
+ *   - Device epochs (sfc_config.device_epochs): the next epoch is a word in
+ *     device memory that each launch reads when it starts and that its last
+ *     warp advances when every warp has finished, so a call enqueued now
+ *     takes whatever epoch the stream order gives it. Calls must pass epoch 0
+ *     (any other value: SFC_ERR_EPOCH), sfc_next_epoch returns 0,
+ *     sfc_reserve_epochs is unsupported and sfc_reset sets the word back
+ *     to 1. This makes calls capturable in a CUDA graph and replayable: each
+ *     replay continues the sequence. A launch whose epochs would pass
+ *     2^32 - 1 records SFC_ERR_EPOCH instead of running.
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*,
  *     NULL = the legacy default stream). Calls on one context must be
  *     ordered on the GPU (one stream, or streams joined by events).
@@ -110,6 +119,8 @@ typedef struct {
   uint32_t timeout_us;      /* bound on each device-side wait; 0 = 50000 */
   int debug_checks;         /* nonzero: the kernel rejects sentinel inputs */
   uint32_t protocol_mask;   /* bit p provisions scratch for protocol p; 0 = all */
+  int device_epochs;        /* nonzero: the epoch sequence lives on the device
+                               (calls pass epoch 0; CUDA-graph replayable) */
 } sfc_config;
 
 /* Latency model of the selector, one entry per (op, protocol, nranks):

@@ -18,7 +18,7 @@ SFC_MAX_RANKS = 8
 
 class Config(C.Structure):
     _fields_ = [("ctas_per_rank", C.c_int), ("timeout_us", C.c_uint32), ("debug_checks", C.c_int),
-                ("protocol_mask", C.c_uint32)]
+                ("protocol_mask", C.c_uint32), ("device_epochs", C.c_int)]
 
 
 SFC_COST_BUCKETS = 24

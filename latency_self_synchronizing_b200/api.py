@@ -117,7 +117,10 @@ class Communicator:
     """N emulated ranks on the current CUDA device (one libsfc context)."""
 
     def __init__(self, nranks, max_bytes_per_rank, *, ctas_per_rank=0, timeout_us=0, debug_checks=False,
-                 protocols=None):
+                 protocols=None, device_epochs=False):
+        """device_epochs=True keeps the epoch sequence on the device: calls
+        take no epoch, next_epoch reads 0, and calls can be captured in a
+        CUDA graph and replayed (each replay continues the sequence)."""
         if not torch.cuda.is_available():
             raise RuntimeError("a CUDA device is required")
         self._lib = _lib.load()
@@ -125,7 +128,7 @@ class Communicator:
         if protocols is not None:
             for p in protocols:
                 mask |= 1 << int(as_protocol(p))
-        cfg = _lib.Config(int(ctas_per_rank), int(timeout_us), int(bool(debug_checks)), mask)
+        cfg = _lib.Config(int(ctas_per_rank), int(timeout_us), int(bool(debug_checks)), mask, int(bool(device_epochs)))
         handle = C.c_void_p()
         torch.cuda.init()
         _check(self._lib.sfc_init(C.byref(handle), int(nranks), int(max_bytes_per_rank), C.byref(cfg)), "sfc_init")
@@ -229,7 +232,7 @@ class Communicator:
             if timings.dtype != torch.int64 or timings.numel() < k_ops + 1:
                 raise ValueError("timings must be an int64 CUDA tensor of k_ops + 1 entries")
             tim_p = C.c_void_p(timings.data_ptr())
-        e = self.next_epoch if epoch is None else int(epoch)
+        e = 0 if epoch is None else int(epoch)  # 0 = the next epoch
         _check(fn(self._ctx, int(k_ops), C.c_void_p(in_table.data_ptr()), C.c_void_p(out_table.data_ptr()),
                   int(count), 0, int(as_protocol(protocol)), e, skew_p, tim_p, _stream_handle(stream)),
                fn.__name__)
@@ -254,7 +257,7 @@ class Communicator:
         if n != self.nranks or tuple(out_host.shape) != (k, n, count):
             raise ValueError("shape mismatch")
         tim_p = None if timings is None else C.c_void_p(timings.data_ptr())
-        e = self.next_epoch if epoch is None else int(epoch)
+        e = 0 if epoch is None else int(epoch)  # 0 = the next epoch
         _check(self._lib.sfc_allreduce_chain_host(self._ctx, int(k), C.c_void_p(in_host.data_ptr()),
                                                   C.c_void_p(out_host.data_ptr()), int(count), 0,
                                                   int(as_protocol(protocol)), e, tim_p, _stream_handle(stream)),
@@ -274,7 +277,7 @@ class Communicator:
         W = (C.c_void_p * n)(*[_dev_ptr(w, "weight") for w in weights])
         X = (C.c_void_p * n)(*[_dev_ptr(t, "input") for t in xs])
         Y = (C.c_void_p * n)(*[_dev_ptr(t, "output") for t in ys])
-        e = self.next_epoch if epoch is None else int(epoch)
+        e = 0 if epoch is None else int(epoch)  # 0 = the next epoch
         _check(self._lib.sfc_linear_allreduce(self._ctx, W, X, Y, int(hidden), int(kdim), e, _stream_handle(stream)),
                "sfc_linear_allreduce")
 

@@ -83,6 +83,22 @@ SFC_DEV uint64_t atom_exch_u64(void* p, uint64_t v) {
   asm volatile("atom.relaxed.gpu.global.exch.b64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
   return old;
 }
+// Device-epoch mode: the epoch this launch starts at. Written by the
+// previous launch's last warp; the kernel boundary makes it visible.
+SFC_DEV uint32_t device_epoch(const uint32_t* w) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(w) : "memory");
+  return v;
+}
+// Lane 0 of every warp that finished its launch counts itself; the last of
+// `warps` resets the counter and publishes the next epoch.
+SFC_DEV void finish_device_epoch(uint32_t* epoch_dev, uint32_t* done, uint32_t warps, uint32_t next) {
+  __threadfence();
+  if (atomicAdd(done, 1u) == warps - 1) {
+    atomicExch(done, 0u);
+    atomicExch(epoch_dev, next);
+  }
+}
 // ---- release / acquire -----------------------------------------------------
 SFC_DEV void st_rel_u64(void* p, uint64_t v) {
   asm volatile("st.release.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");

@@ -83,6 +83,14 @@ __global__ void __launch_bounds__(kLinearThreads, 2) linear_allreduce_kernel(con
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint64_t kdim = p.kdim, kvec = kdim / 8, nvec = p.hidden / 8;
   const uint32_t per = p.per_cta, ks = p.ks;
+  const uint32_t epoch = p.epoch_dev != nullptr ? device_epoch(p.epoch_dev) : p.epoch;
+  if (epoch == 0 || epoch == 0xFFFFFFFFu) {  // device epochs ran out: sfc_reset first
+    if (threadIdx.x == 0) {
+      if (atomicCAS(p.view.status, 0, static_cast<int>(SFC_ERR_EPOCH)) == 0) atomicExch(p.view.status + 1, 0);
+      atomicExch(p.view.status + 2, 1);
+    }
+    return;
+  }
   const uint64_t v0 = static_cast<uint64_t>(k) * per;
   const uint64_t v1 = v0 + per < nvec ? v0 + per : nvec;
   const uint32_t owned = v0 < v1 ? static_cast<uint32_t>(v1 - v0) : 0u;
@@ -132,7 +140,7 @@ __global__ void __launch_bounds__(kLinearThreads, 2) linear_allreduce_kernel(con
         const uint4 own = make_uint4(pack_rn(y[0], y[1]), pack_rn(y[2], y[3]), pack_rn(y[4], y[5]),
                                      pack_rn(y[6], y[7]));
         ownv[t] = own;
-        sfc_device::ll_push(p.view, r, p.epoch, v0 + t, own);
+        sfc_device::ll_push(p.view, r, epoch, v0 + t, own);
       }
     }
   }
@@ -142,9 +150,11 @@ __global__ void __launch_bounds__(kLinearThreads, 2) linear_allreduce_kernel(con
     const bool act = t < owned;
     const uint4 own = act ? ownv[t] : make_uint4(0, 0, 0, 0);
     uint4 out;
-    if (!sfc_device::ll_allreduce_lane<NR>(p.view, r, p.epoch, v0 + t, act, own, &out)) return;
+    if (!sfc_device::ll_allreduce_lane<NR>(p.view, r, epoch, v0 + t, act, own, &out)) return;
     if (act) *reinterpret_cast<uint4*>(p.y[r] + (v0 + t) * 8) = out;
   }
+  if (p.epoch_dev != nullptr && lane == 0)
+    finish_device_epoch(p.epoch_dev, p.done_ctr, gridDim.x * (blockDim.x >> 5), epoch + 1);
 }
 
 struct LinearTable {

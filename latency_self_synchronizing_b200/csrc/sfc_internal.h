@@ -90,6 +90,8 @@ struct KParams {
   uint64_t red_stride;  // elements
 
   DevStatus* status;
+  uint32_t* epoch_dev;  // device-epoch mode: the next epoch (read at start), else null
+  uint32_t* done_ctr;   // device-epoch mode: warps finished (the last one advances epoch_dev)
   uint64_t* timings;    // [timing_first + k_ops + 1] or null
   uint32_t timing_first;  // completion of op k is stamped at timings[1 + timing_first + k]
   const uint32_t* skew; // [k_ops * N] ns or null
@@ -108,6 +110,8 @@ struct LinearParams {
   int G;                         // CTAs per rank
   uint32_t epoch;
   uint32_t per_cta;              // output vectors per CTA
+  uint32_t* epoch_dev;           // device-epoch mode (as in KParams), else null
+  uint32_t* done_ctr;
   uint32_t ks;                   // warps that split one vector's columns (1, 2, 4 or 8)
   sfc_ll_view view;
 };

@@ -920,11 +920,19 @@ __global__ void __launch_bounds__(kThreads, MinBlocks<N, PROTO>::value) sfc_kern
   const uint64_t gstride = static_cast<uint64_t>(p.G) * blockDim.x;
   const int lane = threadIdx.x & 31;
   if (ld_rlx_s32(&p.status->abort)) return;  // poisoned context: do nothing
+  uint32_t first = p.first_epoch;
+  if (p.epoch_dev != nullptr) {
+    first = device_epoch(p.epoch_dev);
+    if (first == 0 || static_cast<uint64_t>(first) + p.k_ops - 1 > 0xFFFFFFFFull) {
+      if (threadIdx.x == 0) record_error(p, 4 /* SFC_ERR_EPOCH */, first);
+      return;
+    }
+  }
   if (p.timings != nullptr && lane == 0)
     atomicMin(reinterpret_cast<unsigned long long*>(&p.timings[0]), static_cast<unsigned long long>(gtimer()));
   Operands io{in_ptr<N>(p, 0, r), out_ptr<N>(p, 0, r), nullptr};
   for (int op = 0; op < p.k_ops; ++op) {
-    const uint32_t e = p.first_epoch + static_cast<uint32_t>(op);
+    const uint32_t e = first + static_cast<uint32_t>(op);
     io.in_next = op + 1 < p.k_ops ? in_ptr<N>(p, op + 1, r) : nullptr;
     uint16_t* out_next = op + 1 < p.k_ops ? out_ptr<N>(p, op + 1, r) : nullptr;
     if (p.skew != nullptr) spin_ns(__ldg(&p.skew[op * N + r]), p.timeout_ns);
@@ -954,6 +962,8 @@ __global__ void __launch_bounds__(kThreads, MinBlocks<N, PROTO>::value) sfc_kern
       atomicMax(reinterpret_cast<unsigned long long*>(&p.timings[1 + p.timing_first + op]),
                 static_cast<unsigned long long>(gtimer()));
   }
+  if (p.epoch_dev != nullptr && lane == 0)
+    finish_device_epoch(p.epoch_dev, p.done_ctr, gridDim.x * (blockDim.x >> 5), first + p.k_ops);
 }
 
 // ============================================================ dispatch table

@@ -35,6 +35,8 @@ struct sfc_ctx {
   DevStatus* hstatus = nullptr;  // page-locked mirror
 
   uint32_t next_epoch = 1;
+  uint32_t* d_epoch = nullptr;   // device-epoch mode: {next epoch, finished warps} on the device
+  uint32_t* h_epoch_init = nullptr;  // page-locked {1, 0}, copied over d_epoch by sfc_reset
   bool poisoned = false;
   int silent_rank = -1;
   cudaStream_t last_stream = nullptr;
@@ -148,6 +150,7 @@ sfc_status check_common(sfc_ctx* c, sfc_op op, size_t count, sfc_dtype dtype, in
   if (!provisioned(c, proto)) return SFC_ERR_UNSUPPORTED;
   if (count > c->max_count) return SFC_ERR_INVALID;
   if (c->poisoned) return SFC_ERR_ABORTED;
+  if (c->cfg.device_epochs) return first_epoch == 0 ? SFC_OK : SFC_ERR_EPOCH;  // the kernel checks the range
   if (first_epoch != c->next_epoch) return SFC_ERR_EPOCH;
   if (static_cast<uint64_t>(first_epoch) + static_cast<uint64_t>(k_ops) - 1 > 0xFFFFFFFFull) return SFC_ERR_EPOCH;
   return SFC_OK;
@@ -161,6 +164,8 @@ void fill_common(sfc_ctx* c, KParams& p, int proto, uint64_t count, int k_ops, u
   p.scratch = self_sync(proto) ? c->region[proto] : nullptr;
   p.slot_stride = self_sync(proto) ? c->slot_stride[proto] : 0;
   p.scratch_bytes = self_sync(proto) ? c->region_bytes[proto] : 0;
+  p.epoch_dev = c->cfg.device_epochs ? c->d_epoch : nullptr;
+  p.done_ctr = c->cfg.device_epochs ? c->d_epoch + 1 : nullptr;
   p.bar = c->bar;
   p.bar_stride = c->bar_stride;
   p.red = c->red;
@@ -198,7 +203,8 @@ sfc_status prepare_timings(uint64_t* timings, int k_ops, cudaStream_t stream) {
 }
 
 // Epoch 0 is never a valid epoch; callers pass it for "the next one".
-uint32_t resolve_epoch(const sfc_ctx* c, uint32_t e) { return e == 0 ? c->next_epoch : e; }
+// (In device-epoch mode 0 stays 0: the kernel reads the epoch.)
+uint32_t resolve_epoch(const sfc_ctx* c, uint32_t e) { return e == 0 && !c->cfg.device_epochs ? c->next_epoch : e; }
 
 sfc_status one_op(sfc_ctx* c, sfc_op op, const void* const* in, void* const* out, size_t count, sfc_dtype dtype,
                   sfc_protocol protocol, uint32_t epoch, void* stream) {
@@ -230,7 +236,7 @@ sfc_status one_op(sfc_ctx* c, sfc_op op, const void* const* in, void* const* out
   const int G = choose_G(c, proto, op, count, nullptr);
   fill_common(c, p, proto, count, 1, epoch, G);
   s = launch(c, proto, op, p, static_cast<cudaStream_t>(stream));
-  if (s == SFC_OK) c->next_epoch = epoch + 1;
+  if (s == SFC_OK && !c->cfg.device_epochs) c->next_epoch = epoch + 1;
   return s;
 }
 
@@ -257,7 +263,7 @@ sfc_status chain(sfc_ctx* c, sfc_op op, int k_ops, const void* const* in_table, 
   const int G = choose_G(c, proto, op, count, nullptr);
   fill_common(c, p, proto, count, k_ops, first_epoch, G);
   s = launch(c, proto, op, p, st);
-  if (s == SFC_OK) c->next_epoch = first_epoch + static_cast<uint32_t>(k_ops);
+  if (s == SFC_OK && !c->cfg.device_epochs) c->next_epoch = first_epoch + static_cast<uint32_t>(k_ops);
   return s;
 }
 
@@ -501,6 +507,11 @@ sfc_status sfc_init(sfc_ctx** out, int nranks, size_t max_bytes_per_rank, const 
   }
   if (!cuda_ok(cudaMalloc(&c->dstatus, sizeof(DevStatus)))) return fail(SFC_ERR_CUDA);
   if (!cuda_ok(cudaMallocHost(&c->hstatus, sizeof(DevStatus)))) return fail(SFC_ERR_CUDA);
+  if (!cuda_ok(cudaMalloc(&c->d_epoch, 2 * sizeof(uint32_t))) ||
+      !cuda_ok(cudaMallocHost(&c->h_epoch_init, 2 * sizeof(uint32_t))))
+    return fail(SFC_ERR_CUDA);
+  c->h_epoch_init[0] = 1;
+  c->h_epoch_init[1] = 0;
   sfc_status s = sfc_reset(c, nullptr);
   if (s != SFC_OK) return fail(s);
   if (!cuda_ok(cudaStreamSynchronize(nullptr))) return fail(SFC_ERR_CUDA);
@@ -520,6 +531,8 @@ sfc_status sfc_destroy(sfc_ctx* c) {
   if (c->red) cudaFree(c->red);
   if (c->dstatus) cudaFree(c->dstatus);
   if (c->hstatus) cudaFreeHost(c->hstatus);
+  if (c->d_epoch) cudaFree(c->d_epoch);
+  if (c->h_epoch_init) cudaFreeHost(c->h_epoch_init);
   if (c->stage_in) cudaFree(c->stage_in);
   if (c->stage_out) cudaFree(c->stage_out);
   if (c->h2d) cudaStreamDestroy(c->h2d);
@@ -542,6 +555,8 @@ sfc_status sfc_reset(sfc_ctx* c, void* stream) {
   }
   if (!cuda_ok(cudaMemsetAsync(c->bar, 0, sizeof(uint64_t) * c->nranks * c->bar_stride, st))) return SFC_ERR_CUDA;
   if (!cuda_ok(cudaMemsetAsync(c->dstatus, 0, sizeof(DevStatus), st))) return SFC_ERR_CUDA;
+  if (!cuda_ok(cudaMemcpyAsync(c->d_epoch, c->h_epoch_init, 2 * sizeof(uint32_t), cudaMemcpyHostToDevice, st)))
+    return SFC_ERR_CUDA;
   c->next_epoch = 1;
   c->poisoned = false;
   c->last_stream = st;
@@ -658,7 +673,7 @@ sfc_status sfc_allreduce_chain_host(sfc_ctx* c, int k_ops, const void* in_host, 
     fill_common(c, p, proto, count, kj, first_epoch + static_cast<uint32_t>(a), G);
     s = launch(c, proto, SFC_OP_ALLREDUCE, p, st);
     if (s != SFC_OK) return s;
-    c->next_epoch = first_epoch + static_cast<uint32_t>(a + kj);
+    if (!c->cfg.device_epochs) c->next_epoch = first_epoch + static_cast<uint32_t>(a + kj);
     if (!cuda_ok(cudaEventRecord(c->ev_run[j], st)) || !cuda_ok(cudaStreamWaitEvent(c->d2h, c->ev_run[j], 0)) ||
         !copy(static_cast<uint8_t*>(out_host) + row0 * row_host, row_host, c->stage_out + row0 * stride, row_dev,
               rows, cudaMemcpyDeviceToHost, c->d2h) ||
@@ -681,7 +696,7 @@ sfc_status sfc_get_status(sfc_ctx* c, uint32_t* info) {
   return static_cast<sfc_status>(code);
 }
 
-uint32_t sfc_next_epoch(const sfc_ctx* c) { return c ? c->next_epoch : 0; }
+uint32_t sfc_next_epoch(const sfc_ctx* c) { return c && !c->cfg.device_epochs ? c->next_epoch : 0; }
 
 sfc_status sfc_launch_shape(sfc_ctx* c, sfc_op op, sfc_protocol protocol, size_t count, int* ctas_per_rank,
                             int* threads_per_cta) {
@@ -735,6 +750,7 @@ sfc_status sfc_get_ll_view(sfc_ctx* c, sfc_ll_view* view) {
 
 sfc_status sfc_reserve_epochs(sfc_ctx* c, uint32_t k, uint32_t* first) {
   if (c == nullptr || first == nullptr || k == 0) return SFC_ERR_INVALID;
+  if (c->cfg.device_epochs) return SFC_ERR_UNSUPPORTED;  // the host does not know the epoch
   if (c->poisoned) return SFC_ERR_ABORTED;
   if (static_cast<uint64_t>(c->next_epoch) + k - 1 > 0xFFFFFFFFull) return SFC_ERR_EPOCH;
   *first = c->next_epoch;
@@ -750,9 +766,11 @@ sfc_status sfc_linear_allreduce(sfc_ctx* c, const void* const* W, const void* co
   if (c->region[kLL] == nullptr) return SFC_ERR_UNSUPPORTED;
   if (c->poisoned) return SFC_ERR_ABORTED;
   epoch = resolve_epoch(c, epoch);
-  if (epoch != c->next_epoch) return SFC_ERR_EPOCH;
+  if (c->cfg.device_epochs ? epoch != 0 : epoch != c->next_epoch) return SFC_ERR_EPOCH;
   const int N = c->nranks;
   sfc::LinearParams p{};
+  p.epoch_dev = c->cfg.device_epochs ? c->d_epoch : nullptr;
+  p.done_ctr = c->cfg.device_epochs ? c->d_epoch + 1 : nullptr;
   for (int r = 0; r < N; ++r) {
     if (!W[r] || !x[r] || !y[r] || !aligned16(W[r]) || !aligned16(x[r]) || !aligned16(y[r])) return SFC_ERR_INVALID;
     p.W[r] = static_cast<const uint16_t*>(W[r]);
@@ -818,7 +836,7 @@ sfc_status sfc_linear_allreduce(sfc_ctx* c, const void* const* W, const void* co
   if (!cuda_ok(e)) return SFC_ERR_CUDA;
   c->launches++;
   c->last_stream = st;
-  c->next_epoch = epoch + 1;
+  if (!c->cfg.device_epochs) c->next_epoch = epoch + 1;
   return SFC_OK;
 }
 
