@@ -113,6 +113,7 @@ extern "C" sfc_status sfc_allreduce_noalloc(const void* const* in, void* const* 
   p.first_epoch = 1;
   p.scratch = base;
   p.slot_stride = slot;
+  p.scratch_bytes = used;
   p.status = reinterpret_cast<DevStatus*>(status);
   p.timeout_ns = 50ull * 1000 * 1000;
   p.silent_rank = -1;
