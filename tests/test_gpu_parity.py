@@ -320,3 +320,34 @@ def test_cta_size_boundary(comms, proto, n):
         _assert_ar(run_chain(comm, proto, x), x)
         xg = make_inputs(seed=count + n + 1, k_ops=2, nranks=n, count=count // n)
         _assert_ag(run_chain(comm, proto, xg, op="allgather"), xg)
+
+
+SPECIAL = np.array([0x0000, 0x8000, 0x0001, 0x8001, 0x007F, 0x807F, 0x0080, 0x8080, 0x7F7F, 0xFF7F, 0x7F00,
+                    0xFF00, 0x3F80, 0xBF80, 0x7F80, 0xFF80], dtype=np.uint16)
+
+
+def _special_inputs(seed, k, n, count):
+    """bf16 edge values: signed zeros, subnormals (lost if anything flushed
+    them), the smallest normal, the largest finite values (sums overflow to
+    inf), infinities. An element with an infinite input gets only +inf and
+    no large negative value, so no element meets +inf and -inf (a NaN, whose
+    payload is not compared)."""
+    rng = np.random.default_rng(seed)
+    x = SPECIAL[rng.integers(0, len(SPECIAL), size=(k, n, count))]
+    has_inf = np.broadcast_to(((x == 0x7F80) | (x == 0xFF80)).any(axis=1)[:, None, :], x.shape)
+    x = np.where(has_inf & (x == 0xFF80), np.uint16(0x7F80), x)
+    x = np.where(has_inf & ((x == 0xFF7F) | (x == 0xFF00)), np.uint16(0xBF80), x)
+    return x
+
+
+@pytest.mark.parametrize("proto", AR_PROTOS)
+@pytest.mark.parametrize("n", [2, 3, 8])
+def test_special_values_bit_exact(comms, proto, n):
+    comm = comms(n)
+    x = _special_inputs(seed=n * 31, k=2, n=n, count=4099)
+    want = _want_ar(x)
+    assert not np.any((want & 0x7FFF) > 0x7F80), "test inputs must not produce NaN"
+    # the cases are present: subnormal or zero results, infinities, and -0 (n = 2)
+    assert np.any((want & 0x7F80) == 0) and np.any((want & 0x7FFF) == 0x7F80)
+    assert n != 2 or np.any(want == 0x8000)
+    _assert_ar(run_chain(comm, proto, x), x)
