@@ -77,6 +77,8 @@ SIGNATURES = [
     ("sfc_reserve_epochs", _S, [_P, C.c_uint32, C.POINTER(C.c_uint32)]),
     ("sfc_linear_allreduce", _S, [_P, C.POINTER(_P), C.POINTER(_P), C.POINTER(_P), C.c_size_t, C.c_size_t,
                                   C.c_uint32, _P]),
+    ("sfc_linear_allreduce_tokens", _S, [_P, C.POINTER(_P), C.POINTER(_P), C.POINTER(_P), C.c_size_t, C.c_size_t,
+                                          C.c_uint32, C.c_uint32, _P]),
     ("sfc_allreduce_noalloc", _S, [C.POINTER(_P), C.POINTER(_P), C.c_int, C.c_size_t, _P]),
 ]
 

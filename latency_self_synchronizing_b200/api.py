@@ -264,22 +264,24 @@ class Communicator:
                "sfc_allreduce_chain_host")
 
     def linear_allreduce(self, weights, xs, ys, epoch=None, stream=None):
-        """Fused row-parallel linear + all-reduce for one token:
+        """Fused row-parallel linear + all-reduce for 1..8 decode tokens:
         ys[r] = sum over ranks of bf16(weights[q] @ xs[q]) (rank order, one
-        rounding), weights[r] [hidden, kdim], xs[r] [kdim], ys[r] [hidden]."""
+        rounding); weights[r] [hidden, kdim]; xs[r] [kdim] (one token) or
+        [tokens, kdim]; ys[r] [hidden] or [tokens, hidden], matching xs."""
         n = self.nranks
         if not (len(weights) == len(xs) == len(ys) == n):
             raise ValueError(f"need {n} weights, inputs and outputs")
         hidden, kdim = weights[0].shape
+        tokens = 1 if xs[0].dim() == 1 else int(xs[0].shape[0])
         for w, x_, y_ in zip(weights, xs, ys):
-            if tuple(w.shape) != (hidden, kdim) or x_.numel() != kdim or y_.numel() != hidden:
+            if tuple(w.shape) != (hidden, kdim) or x_.numel() != tokens * kdim or y_.numel() != tokens * hidden:
                 raise ValueError("shape mismatch")
         W = (C.c_void_p * n)(*[_dev_ptr(w, "weight") for w in weights])
         X = (C.c_void_p * n)(*[_dev_ptr(t, "input") for t in xs])
         Y = (C.c_void_p * n)(*[_dev_ptr(t, "output") for t in ys])
         e = 0 if epoch is None else int(epoch)  # 0 = the next epoch
-        _check(self._lib.sfc_linear_allreduce(self._ctx, W, X, Y, int(hidden), int(kdim), e, _stream_handle(stream)),
-               "sfc_linear_allreduce")
+        _check(self._lib.sfc_linear_allreduce_tokens(self._ctx, W, X, Y, int(hidden), int(kdim), tokens, e,
+                                                     _stream_handle(stream)), "sfc_linear_allreduce_tokens")
 
     def ll_view(self):
         v = _lib.LLView()

@@ -1,4 +1,4 @@
-// Row-parallel linear layer fused with its all-reduce, for one decode token
+// Row-parallel linear layer fused with its all-reduce, for 1..8 decode tokens
 // (the tensor-parallel decode pattern "SiFAR: Synchronization-Free All-Reduce
 // for Low-Latency LLM Inference", introduction, and "Why Microseconds Matter
 // in AI Infrastructure", section "Latency can matter more than bandwidth",
@@ -22,6 +22,12 @@
 // the ks parts in part order, rounds to bf16 and pushes the vector to every
 // peer. After the CTA's last vector, all its threads poll their vectors
 // (rank-order fp32 fold, one bf16 rounding) and store y_r.
+//
+// Several tokens (a decode step's batch) share one pass over the weights: a
+// kernel instance carries a token tile T (1, 2, 4 or 8), keeps 8 x T dot
+// products per lane and pushes one vector per (token, 8 rows); token u's
+// vector v is LL vector u * hidden / 8 + v, so the all-reduce covers
+// tokens x hidden elements.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -73,16 +79,19 @@ SFC_DEV float fold8(const float (&a)[8], int lane) {
   return s;
 }
 
-// Shared memory: x_r | parts [per][ks][8] fp32 | own [per] (packed bf16) |
-// counters [per].
-template <int NR>
-__global__ void __launch_bounds__(kLinearThreads, 2) linear_allreduce_kernel(const __grid_constant__ LinearParams p) {
+// Shared memory: x_r [T][kdim] | parts [per][ks][T][8] fp32 |
+// own [per][T] (packed bf16) | counters [per]. T = token tile (1, 2, 4, 8);
+// tokens past p.tokens are zero and never leave the CTA.
+// (8 tokens keep 64 accumulators a lane: one CTA per SM, so nothing spills)
+template <int NR, int T>
+__global__ void __launch_bounds__(kLinearThreads, T >= 8 ? 1 : 2)
+    linear_allreduce_kernel(const __grid_constant__ LinearParams p) {
   extern __shared__ __align__(16) unsigned char sm[];
   const int r = blockIdx.x / p.G;
   const int k = blockIdx.x - r * p.G;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint64_t kdim = p.kdim, kvec = kdim / 8, nvec = p.hidden / 8;
-  const uint32_t per = p.per_cta, ks = p.ks;
+  const uint32_t per = p.per_cta, ks = p.ks, tokens = p.tokens;
   const uint32_t epoch = p.epoch_dev != nullptr ? device_epoch(p.epoch_dev) : p.epoch;
   if (epoch == 0 || epoch == 0xFFFFFFFFu) {  // device epochs ran out: sfc_reset first
     if (threadIdx.x == 0) {
@@ -96,11 +105,14 @@ __global__ void __launch_bounds__(kLinearThreads, 2) linear_allreduce_kernel(con
   const uint32_t owned = v0 < v1 ? static_cast<uint32_t>(v1 - v0) : 0u;
 
   uint4* xs = reinterpret_cast<uint4*>(sm);
-  float* parts = reinterpret_cast<float*>(sm + kdim * 2);
-  uint4* ownv = reinterpret_cast<uint4*>(parts + static_cast<uint64_t>(per) * ks * 8);
-  uint32_t* cnt = reinterpret_cast<uint32_t*>(ownv + per);
+  float* parts = reinterpret_cast<float*>(sm + kdim * 2 * T);
+  uint4* ownv = reinterpret_cast<uint4*>(parts + static_cast<uint64_t>(per) * ks * T * 8);
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(ownv + static_cast<uint64_t>(per) * T);
 
-  for (uint64_t i = threadIdx.x; i < kvec; i += blockDim.x) xs[i] = ld_nc_v4(p.x[r] + i * 8);
+  for (uint64_t i = threadIdx.x; i < kvec * T; i += blockDim.x) {
+    const uint64_t tok = i / kvec;
+    xs[i] = tok < tokens ? ld_nc_v4(p.x[r] + tok * kdim + (i - tok * kvec) * 8) : make_uint4(0, 0, 0, 0);
+  }
   for (uint32_t i = threadIdx.x; i < per; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
 
@@ -109,72 +121,94 @@ __global__ void __launch_bounds__(kLinearThreads, 2) linear_allreduce_kernel(con
   const uint16_t* W = p.W[r];
   for (uint32_t t = g; t < owned; t += groups) {
     const uint16_t* rows = W + (v0 + t) * 8 * kdim;
-    float acc[8];
+    float acc[T][8];
 #pragma unroll
-    for (int m = 0; m < 8; ++m) acc[m] = 0.f;
-#pragma unroll 2
+    for (int u = 0; u < T; ++u)
+#pragma unroll
+      for (int m = 0; m < 8; ++m) acc[u][m] = 0.f;
+    // two chunks' loads in flight up to 4 tokens; at 8 tokens the 64
+    // accumulators leave no room (measured: unrolling there is slower)
+#pragma unroll(T <= 4 ? 2 : 1)
     for (uint64_t c = c_lo + lane; c < c_hi; c += 32) {
-      const uint4 xv = xs[c];
       uint4 wv[8];
 #pragma unroll
       for (int m = 0; m < 8; ++m) wv[m] = ld_stream_v4(rows + m * kdim + c * 8);
 #pragma unroll
-      for (int m = 0; m < 8; ++m) acc[m] = dot8(wv[m], xv, acc[m]);
+      for (int u = 0; u < T; ++u) {
+        const uint4 xv = xs[u * kvec + c];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) acc[u][m] = dot8(wv[m], xv, acc[u][m]);
+      }
     }
-    const float s = fold8(acc, lane);
-    float* pt = parts + (static_cast<uint64_t>(t) * ks + h) * 8;
-    if ((lane & 3) == 0) pt[lane >> 2] = s;
+    float* pt = parts + (static_cast<uint64_t>(t) * ks + h) * T * 8;
+#pragma unroll
+    for (int u = 0; u < T; ++u) {
+      const float s = fold8(acc[u], lane);
+      if ((lane & 3) == 0) pt[u * 8 + (lane >> 2)] = s;
+    }
     __threadfence_block();
     __syncwarp();
     if (lane == 0) {
-      // the last of the group's ks warps completes the vector
+      // the last of the group's ks warps completes the vector (all tokens)
       if (atomicAdd(&cnt[t], 1u) == ks - 1) {
         __threadfence_block();
-        const volatile float* pv = parts + static_cast<uint64_t>(t) * ks * 8;
-        float y[8];
+        const volatile float* pv = parts + static_cast<uint64_t>(t) * ks * T * 8;
+        for (uint32_t u = 0; u < tokens; ++u) {
+          float y[8];
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          y[m] = pv[m];
-          for (uint32_t j = 1; j < ks; ++j) y[m] += pv[j * 8 + m];
+          for (int m = 0; m < 8; ++m) {
+            y[m] = pv[u * 8 + m];
+            for (uint32_t j = 1; j < ks; ++j) y[m] += pv[(j * T + u) * 8 + m];
+          }
+          const uint4 own = make_uint4(pack_rn(y[0], y[1]), pack_rn(y[2], y[3]), pack_rn(y[4], y[5]),
+                                       pack_rn(y[6], y[7]));
+          ownv[t * T + u] = own;
+          sfc_device::ll_push(p.view, r, epoch, u * nvec + v0 + t, own);
         }
-        const uint4 own = make_uint4(pack_rn(y[0], y[1]), pack_rn(y[2], y[3]), pack_rn(y[4], y[5]),
-                                     pack_rn(y[6], y[7]));
-        ownv[t] = own;
-        sfc_device::ll_push(p.view, r, epoch, v0 + t, own);
       }
     }
   }
   __syncthreads();  // every vector of the CTA is pushed and its own part stored
-  for (uint32_t base = 0; base < owned; base += kLinearThreads) {
-    const uint32_t t = base + threadIdx.x;
-    const bool act = t < owned;
-    const uint4 own = act ? ownv[t] : make_uint4(0, 0, 0, 0);
+  const uint32_t work = owned * tokens;
+  for (uint32_t base = 0; base < work; base += kLinearThreads) {
+    const uint32_t i = base + threadIdx.x;
+    const bool act = i < work;
+    const uint32_t u = act ? i / owned : 0, t = act ? i - u * owned : 0;
+    const uint4 own = act ? ownv[t * T + u] : make_uint4(0, 0, 0, 0);
     uint4 out;
-    if (!sfc_device::ll_allreduce_lane<NR>(p.view, r, epoch, v0 + t, act, own, &out)) return;
-    if (act) *reinterpret_cast<uint4*>(p.y[r] + (v0 + t) * 8) = out;
+    if (!sfc_device::ll_allreduce_lane<NR>(p.view, r, epoch, u * nvec + v0 + t, act, own, &out)) return;
+    if (act) *reinterpret_cast<uint4*>(p.y[r] + u * p.hidden + (v0 + t) * 8) = out;
   }
   if (p.epoch_dev != nullptr && lane == 0)
     finish_device_epoch(p.epoch_dev, p.done_ctr, gridDim.x * (blockDim.x >> 5), epoch + 1);
 }
 
-struct LinearTable {
-  const void* t[kMaxRanks + 1] = {};
-  LinearTable() {
-    t[2] = reinterpret_cast<const void*>(&linear_allreduce_kernel<2>);
-    t[3] = reinterpret_cast<const void*>(&linear_allreduce_kernel<3>);
-    t[4] = reinterpret_cast<const void*>(&linear_allreduce_kernel<4>);
-    t[5] = reinterpret_cast<const void*>(&linear_allreduce_kernel<5>);
-    t[6] = reinterpret_cast<const void*>(&linear_allreduce_kernel<6>);
-    t[7] = reinterpret_cast<const void*>(&linear_allreduce_kernel<7>);
-    t[8] = reinterpret_cast<const void*>(&linear_allreduce_kernel<8>);
+template <int NR>
+struct LinearRow {
+  static const void* get(uint32_t T) {
+    switch (T) {
+      case 1: return reinterpret_cast<const void*>(&linear_allreduce_kernel<NR, 1>);
+      case 2: return reinterpret_cast<const void*>(&linear_allreduce_kernel<NR, 2>);
+      case 4: return reinterpret_cast<const void*>(&linear_allreduce_kernel<NR, 4>);
+      case 8: return reinterpret_cast<const void*>(&linear_allreduce_kernel<NR, 8>);
+      default: return nullptr;
+    }
   }
 };
 
 }  // namespace
 
-const void* linear_kernel_for(int nranks) {
-  static const LinearTable table;
-  return (nranks >= kMinRanks && nranks <= kMaxRanks) ? table.t[nranks] : nullptr;
+const void* linear_kernel_for(int nranks, uint32_t token_tile) {
+  switch (nranks) {
+    case 2: return LinearRow<2>::get(token_tile);
+    case 3: return LinearRow<3>::get(token_tile);
+    case 4: return LinearRow<4>::get(token_tile);
+    case 5: return LinearRow<5>::get(token_tile);
+    case 6: return LinearRow<6>::get(token_tile);
+    case 7: return LinearRow<7>::get(token_tile);
+    case 8: return LinearRow<8>::get(token_tile);
+    default: return nullptr;
+  }
 }
 
 }  // namespace sfc

@@ -103,10 +103,11 @@ struct KParams {
 // Fused row-parallel linear + LL all-reduce (one decode token).
 struct LinearParams {
   const uint16_t* W[kMaxRanks];  // [hidden][kdim] row-major, per rank
-  const uint16_t* x[kMaxRanks];  // [kdim], per rank
-  uint16_t* y[kMaxRanks];        // [hidden], per rank
+  const uint16_t* x[kMaxRanks];  // [tokens][kdim], per rank
+  uint16_t* y[kMaxRanks];        // [tokens][hidden], per rank
   uint64_t hidden;
   uint64_t kdim;
+  uint32_t tokens;               // 1..8; the kernel's token tile T is the next power of two
   int G;                         // CTAs per rank
   uint32_t epoch;
   uint32_t per_cta;              // output vectors per CTA
@@ -117,11 +118,15 @@ struct LinearParams {
 };
 constexpr int kLinearThreads = 256;
 constexpr int kLinearWarps = kLinearThreads / 32;
-// dynamic shared memory of the fused kernel: x, per-part sums, own vectors, counters
-inline size_t linear_smem_bytes(uint64_t kdim, uint32_t ks, uint32_t per_cta) {
-  return kdim * 2 + 32ull * ks * per_cta + 16ull * per_cta + 4ull * per_cta;
+constexpr uint32_t kLinearMaxTokens = 8;
+// token tile of the fused kernel for a token count: 1, 2, 4 or 8
+inline uint32_t linear_token_tile(uint32_t tokens) { return tokens <= 1 ? 1 : tokens <= 2 ? 2 : tokens <= 4 ? 4 : 8; }
+// dynamic shared memory of the fused kernel: x (T tokens), per-part sums,
+// own vectors, counters
+inline size_t linear_smem_bytes(uint64_t kdim, uint32_t T, uint32_t ks, uint32_t per_cta) {
+  return kdim * 2 * T + 32ull * ks * T * per_cta + 16ull * T * per_cta + 4ull * per_cta;
 }
-const void* linear_kernel_for(int nranks);
+const void* linear_kernel_for(int nranks, uint32_t token_tile);
 
 // Kernel entry for (nranks, protocol, op); null if not provided.
 const void* kernel_for(int nranks, int protocol, int op);

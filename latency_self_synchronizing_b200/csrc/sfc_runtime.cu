@@ -46,7 +46,7 @@ struct sfc_ctx {
   int occupancy[kNumProtocols][2][2] = {};  // blocks per SM, per (protocol, op, CTA size), 0 = unknown
   int forced_protocol = 0;                // SFC_PROTOCOL: what AUTO resolves to (0 = the selector)
   int smem_optin = 0;                     // opt-in shared memory per block (bytes)
-  int linear_occ = 0;                     // fused-linear CTAs per SM (0 = not yet queried)
+  int linear_occ[4] = {};                 // fused-linear CTAs per SM per token tile 1/2/4/8 (0 = not queried)
 
   // staging for the host-buffer entry point, and the copy streams and
   // events that overlap its copies with the chain segments
@@ -760,8 +760,15 @@ sfc_status sfc_reserve_epochs(sfc_ctx* c, uint32_t k, uint32_t* first) {
 
 sfc_status sfc_linear_allreduce(sfc_ctx* c, const void* const* W, const void* const* x, void* const* y,
                                 size_t hidden, size_t kdim, uint32_t epoch, void* stream) {
+  return sfc_linear_allreduce_tokens(c, W, x, y, hidden, kdim, 1, epoch, stream);
+}
+
+sfc_status sfc_linear_allreduce_tokens(sfc_ctx* c, const void* const* W, const void* const* x, void* const* y,
+                                       size_t hidden, size_t kdim, uint32_t tokens, uint32_t epoch, void* stream) {
   if (c == nullptr || W == nullptr || x == nullptr || y == nullptr) return SFC_ERR_INVALID;
-  if (hidden == 0 || hidden % 8 || hidden > c->max_count || kdim == 0 || kdim % 8 || kdim > 49152)
+  if (tokens < 1 || tokens > sfc::kLinearMaxTokens) return SFC_ERR_INVALID;
+  const uint32_t T = sfc::linear_token_tile(tokens);
+  if (hidden == 0 || hidden % 8 || hidden * tokens > c->max_count || kdim == 0 || kdim % 8 || kdim * T > 49152)
     return SFC_ERR_INVALID;
   if (c->region[kLL] == nullptr) return SFC_ERR_UNSUPPORTED;
   if (c->poisoned) return SFC_ERR_ABORTED;
@@ -777,24 +784,26 @@ sfc_status sfc_linear_allreduce(sfc_ctx* c, const void* const* W, const void* co
     p.x[r] = static_cast<const uint16_t*>(x[r]);
     p.y[r] = static_cast<uint16_t*>(y[r]);
   }
+  const size_t xb = tokens * kdim * 2, yb = tokens * hidden * 2;
   for (int a = 0; a < N; ++a)
     for (int b = 0; b < N; ++b)
-      if (overlap(y[a], hidden * 2, x[b], kdim * 2) || overlap(y[a], hidden * 2, W[b], hidden * kdim * 2) ||
-          (a < b && overlap(y[a], hidden * 2, y[b], hidden * 2)))
+      if (overlap(y[a], yb, x[b], xb) || overlap(y[a], yb, W[b], hidden * kdim * 2) ||
+          (a < b && overlap(y[a], yb, y[b], yb)))
         return SFC_ERR_INVALID;
-  const void* fn = linear_kernel_for(N);
+  const void* fn = linear_kernel_for(N, T);
   // as many CTAs per rank as fit (two per SM), each rank's output vectors
   // split evenly over its CTAs; ks warps share a vector when that evens out
   // the 8 warps' work (every part keeps at least 128 column chunks, four per
   // lane)
   const uint64_t nvec = hidden / 8, kvec = kdim / 8;
-  int occ = c->linear_occ;
+  const int ti = T == 1 ? 0 : T == 2 ? 1 : T == 4 ? 2 : 3;
+  int occ = c->linear_occ[ti];
   if (occ == 0) {
     if (!cuda_ok(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, c->smem_optin)))
       return SFC_ERR_CUDA;
     if (!cuda_ok(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kLinearThreads, 0)) || occ < 1)
       return SFC_ERR_RESOURCES;
-    c->linear_occ = occ = std::min(occ, 2);
+    c->linear_occ[ti] = occ = std::min(occ, 2);
   }
   int G = occ * c->sm_count / N;
   uint32_t per = 0, ks = 1;
@@ -812,16 +821,17 @@ sfc_status sfc_linear_allreduce(sfc_ctx* c, const void* const* W, const void* co
       }
     }
     // both CTAs of an SM must fit: fewer, larger CTAs if not
-    const size_t smem = sfc::linear_smem_bytes(kdim, ks, per);
+    const size_t smem = sfc::linear_smem_bytes(kdim, T, ks, per);
     if (smem <= static_cast<size_t>(c->smem_optin) &&
         (G * N <= c->sm_count || 2 * (smem + 1024) <= static_cast<size_t>(c->smem_optin) + 1024))
       break;
   }
-  const int smem = static_cast<int>(sfc::linear_smem_bytes(kdim, ks, per));
+  const int smem = static_cast<int>(sfc::linear_smem_bytes(kdim, T, ks, per));
   p.per_cta = per;
   p.ks = ks;
   p.hidden = hidden;
   p.kdim = kdim;
+  p.tokens = tokens;
   p.G = G;
   p.epoch = epoch;
   sfc_status s = sfc_get_ll_view(c, &p.view);

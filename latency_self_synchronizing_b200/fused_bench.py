@@ -2,11 +2,12 @@
 pair (a batched matrix-vector product for all ranks, then an all-reduce).
 
     python -m latency_self_synchronizing_b200.fused_bench [--nranks 4] [--hidden 8192]
-        [--kdim 7168] [--iters 50]
+        [--kdim 7168] [--tokens 1] [--iters 50]
 
 Shapes default to a Llama-3.1-70B MLP down projection with 4-way tensor
 parallelism (hidden 8192, intermediate 28672 / 4 = 7168 per rank), one
-decode token. Weights are normal(0, 0.05), drawn on the device by torch's
+decode token (--tokens: 1..8 tokens of a decode step in one call). Weights
+are normal(0, 0.05), drawn on the device by torch's
 seeded generator (timing only; parity is the tests' job). Consecutive calls
 use different copies of the weights (at least 320 MB in all), so no call
 finds its weights in L2 and every call streams them from HBM. Time per
@@ -50,9 +51,10 @@ def main(argv=None):
     ap.add_argument("--nranks", type=int, default=4)
     ap.add_argument("--hidden", type=int, default=8192)
     ap.add_argument("--kdim", type=int, default=7168)
+    ap.add_argument("--tokens", type=int, default=1)
     ap.add_argument("--iters", type=int, default=50)
     a = ap.parse_args(argv)
-    n, hidden, kdim = a.nranks, a.hidden, a.kdim
+    n, hidden, kdim, tokens = a.nranks, a.hidden, a.kdim, a.tokens
     dev = torch.device("cuda")
     gen = torch.Generator(device=dev)
     gen.manual_seed(0)
@@ -61,16 +63,16 @@ def main(argv=None):
     # their weights in the 126 MB L2 (a decode step's layers are distinct)
     copies = max(2, -(-(320 << 20) // wbytes))
     ws = [(torch.randn(n, hidden, kdim, generator=gen, device=dev) * 0.05).to(torch.bfloat16) for _ in range(copies)]
-    x = torch.randn(n, kdim, 1, generator=gen, device=dev).to(torch.bfloat16)
-    y = torch.empty(n, hidden, dtype=torch.bfloat16, device=dev)
-    part = torch.empty(n, hidden, 1, dtype=torch.bfloat16, device=dev)
-    y2 = torch.empty(n, hidden, dtype=torch.bfloat16, device=dev)
-    comm = api.Communicator(n, hidden * 2)
+    x = torch.randn(n, tokens, kdim, generator=gen, device=dev).to(torch.bfloat16)
+    y = torch.empty(n, tokens, hidden, dtype=torch.bfloat16, device=dev)
+    part = torch.empty(n, tokens, hidden, dtype=torch.bfloat16, device=dev)
+    y2 = torch.empty(n, tokens, hidden, dtype=torch.bfloat16, device=dev)
+    comm = api.Communicator(n, tokens * hidden * 2)
     Ws = [[w[r] for r in range(n)] for w in ws]
-    X = [x[r, :, 0] for r in range(n)]
-    Y = [y[r] for r in range(n)]
-    P = [part[r, :, 0] for r in range(n)]
-    Y2 = [y2[r] for r in range(n)]
+    X = [x[r] if tokens > 1 else x[r, 0] for r in range(n)]
+    Y = [y[r] if tokens > 1 else y[r, 0] for r in range(n)]
+    P = [part[r].view(-1) for r in range(n)]
+    Y2 = [y2[r].view(-1) for r in range(n)]
     turn = [0]
 
     def fused():
@@ -79,7 +81,7 @@ def main(argv=None):
 
     def unfused():
         turn[0] = (turn[0] + 1) % copies
-        torch.bmm(ws[turn[0]], x, out=part)
+        torch.bmm(x, ws[turn[0]].transpose(1, 2), out=part)
         comm.allreduce(P, Y2, protocol="auto")
 
     t_f = _events(fused, a.iters)
@@ -93,9 +95,10 @@ def main(argv=None):
                                                  "MEASURED_PEAKS.json")))["hbm_gbs"])
     except (OSError, KeyError, ValueError):
         pass
-    print(json.dumps({"nranks": n, "hidden": hidden, "kdim": kdim, "weight_copies": copies, "fused_us": t_f,
+    print(json.dumps({"nranks": n, "hidden": hidden, "kdim": kdim, "tokens": tokens, "weight_copies": copies,
+                      "fused_us": t_f,
                       "unfused_us": t_u,
-                      "unfused_selected_protocol": comm.select_protocol("allreduce", hidden * 2).name.lower(),
+                      "unfused_selected_protocol": comm.select_protocol("allreduce", tokens * hidden * 2).name.lower(),
                       "fused_weight_gbs": wbytes / (t_f * 1e-6) / 1e9, "hbm_peak_gbs": peak,
                       "fused_frac": wbytes / (t_f * 1e-6) / 1e9 / peak}))
     comm.close()

@@ -83,3 +83,36 @@ def test_linear_allreduce_shares_the_epoch_sequence():
         assert view.nranks == n and view.slot_stride > 0
     finally:
         comm.close()
+
+
+# several decode tokens in one pass over the weights (token tiles 2, 4, 8;
+# 3, 5, 6, 7 tokens run in the next tile with the extra tokens masked)
+@pytest.mark.parametrize("n,hidden,kdim,tokens", [(2, 64, 512, 2), (4, 8192, 3584, 4), (8, 1024, 1024, 8),
+                                                  (3, 2056, 136, 3), (4, 512, 4096, 5), (2, 1000, 2048, 7),
+                                                  (8, 64, 8, 6), (5, 8192, 1024, 8)])
+def test_linear_allreduce_tokens_within_bound(n, hidden, kdim, tokens):
+    w, _ = _case(n, hidden, kdim, seed=hidden * 3 + kdim + n + tokens)
+    x = make_inputs(seed=hidden + tokens, k_ops=1, nranks=n, count=tokens * kdim, dist="normal",
+                    params=(1.0,))[0].reshape(n, tokens, kdim)
+    comm = api.Communicator(n, tokens * hidden * 2, protocols=["ll"])
+    try:
+        W = [_bf16_dev(w[r]) for r in range(n)]
+        X = [_bf16_dev(x[r]) for r in range(n)]
+        Y = [torch.empty(tokens, hidden, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+        for _ in range(2):
+            comm.linear_allreduce(W, X, Y)
+            torch.cuda.synchronize()
+            assert comm.status()[0] == api.Status.OK
+            ys = [Y[r].cpu().view(torch.int16).numpy().view(np.uint16) for r in range(n)]
+            for r in range(1, n):
+                np.testing.assert_array_equal(ys[r], ys[0])
+            wf = bf16_bits_to_f32(w).astype(np.float64)
+            xf = bf16_bits_to_f32(x).astype(np.float64)
+            d = np.einsum("rhk,rtk->rth", wf, xf)
+            a = np.einsum("rhk,rtk->rth", np.abs(wf), np.abs(xf))
+            eps = 2.0 ** -8 * np.abs(d) + kdim * 2.0 ** -24 * a
+            bound = eps.sum(0) + 2.0 ** -7 * n * (np.abs(d) + eps).sum(0)
+            got = bf16_bits_to_f32(ys[0]).astype(np.float64)
+            assert np.all(np.abs(got - d.sum(0)) <= bound)
+    finally:
+        comm.close()
