@@ -46,15 +46,20 @@ SFC_DEV uint4 ld_stream_v4(const void* p) {
   return v;
 }
 
+// acc + w0 x0 + w1 x1 + ... + w7 x7, one fp32 FMA per element in element
+// order, each taking its two bf16 operands as they are (sm_100's mixed
+// bf16 x bf16 + f32 FMA: the same exact-product, single-rounding step as
+// widening both to f32 first, without the widening instructions).
 SFC_DEV float dot8(uint4 w, uint4 x, float acc) {
-  acc = fmaf(bf_lo(w.x), bf_lo(x.x), acc);
-  acc = fmaf(bf_hi(w.x), bf_hi(x.x), acc);
-  acc = fmaf(bf_lo(w.y), bf_lo(x.y), acc);
-  acc = fmaf(bf_hi(w.y), bf_hi(x.y), acc);
-  acc = fmaf(bf_lo(w.z), bf_lo(x.z), acc);
-  acc = fmaf(bf_hi(w.z), bf_hi(x.z), acc);
-  acc = fmaf(bf_lo(w.w), bf_lo(x.w), acc);
-  acc = fmaf(bf_hi(w.w), bf_hi(x.w), acc);
+  asm("{\n\t.reg .b16 w0, w1, w2, w3, w4, w5, w6, w7, x0, x1, x2, x3, x4, x5, x6, x7;\n\t"
+      "mov.b32 {w0, w1}, %1;\n\tmov.b32 {w2, w3}, %2;\n\tmov.b32 {w4, w5}, %3;\n\tmov.b32 {w6, w7}, %4;\n\t"
+      "mov.b32 {x0, x1}, %5;\n\tmov.b32 {x2, x3}, %6;\n\tmov.b32 {x4, x5}, %7;\n\tmov.b32 {x6, x7}, %8;\n\t"
+      "fma.rn.f32.bf16 %0, w0, x0, %0;\n\tfma.rn.f32.bf16 %0, w1, x1, %0;\n\t"
+      "fma.rn.f32.bf16 %0, w2, x2, %0;\n\tfma.rn.f32.bf16 %0, w3, x3, %0;\n\t"
+      "fma.rn.f32.bf16 %0, w4, x4, %0;\n\tfma.rn.f32.bf16 %0, w5, x5, %0;\n\t"
+      "fma.rn.f32.bf16 %0, w6, x6, %0;\n\tfma.rn.f32.bf16 %0, w7, x7, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(w.x), "r"(w.y), "r"(w.z), "r"(w.w), "r"(x.x), "r"(x.y), "r"(x.z), "r"(x.w));
   return acc;
 }
 
