@@ -142,3 +142,43 @@ def test_one_load_ll128_is_opt_in():
     assert all(t_fast < api.cost_estimate(m, op, p, b, n) for p in ("ll", "ll128", "sentinel"))
     assert api.select_protocol_model(m, op, b, n) == api.Protocol.LL128_FAST
 
+
+
+def _prototypes():
+    """name -> parameter count of every function the header declares."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(sfc_[a-z_0-9]+)\s*\(([^;{]*?)\)\s*;", text):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_the_header():
+    """Every ctypes signature has as many arguments as the C prototype."""
+    protos = _prototypes()
+    for name, _, args in _lib.SIGNATURES:
+        assert name in protos, name
+        assert len(args) == protos[name], (name, len(args), protos[name])
+
+
+def _struct_fields(name):
+    """Member names of `typedef struct { ... } name;` in declaration order."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    m = re.search(r"typedef struct \{([^}]*)\}\s*" + name + r";", text)
+    assert m, name
+    names = []
+    for decl in m.group(1).split(";"):
+        decl = re.sub(r"\[[^\]]*\]", "", decl).strip()
+        if decl:
+            first, *rest = decl.split(",")
+            names.append(first.split()[-1].lstrip("*"))
+            names += [r.strip().lstrip("*") for r in rest]
+    return names
+
+
+@pytest.mark.parametrize("cname,pyname", [("sfc_config", "Config"), ("sfc_cost_entry", "CostEntry"),
+                                           ("sfc_floor_result", "FloorResult"), ("sfc_ll_view", "LLView")])
+def test_binding_structs_match_the_header(cname, pyname):
+    py = [f[0] for f in getattr(_lib, pyname)._fields_]
+    assert _struct_fields(cname) == py
