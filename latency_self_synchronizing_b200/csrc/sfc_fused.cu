@@ -188,10 +188,154 @@ __global__ void __launch_bounds__(kLinearThreads, T >= 8 ? 1 : 2)
     finish_device_epoch(p.epoch_dev, p.done_ctr, gridDim.x * (blockDim.x >> 5), epoch + 1);
 }
 
+// ---------------------------------------------------------------------------
+// 3..8 tokens on the tensor cores (mma.sync m16n8k16, bf16 in, fp32 out).
+// The tile is 16 rows of W_r (two LL vectors) by 8 token columns (tokens past
+// p.tokens are zero). The k order inside one MMA step is a permutation both
+// operands share, chosen so that every thread reads its weights as two
+// coalesced 8-byte pieces: thread (group g, quad q) takes W[row0 + g][k0 + 4q
+// .. 4q+3] and W[row0 + g + 8][same]; its A registers are (row g, k0+4q..+1),
+// (row g+8, k0+4q..+1), (row g, k0+4q+2..+3), (row g+8, k0+4q+2..+3), which
+// the instruction reads as the logical columns 2q, 2q+1 / 2q+8, 2q+9; its B
+// registers are x[token g][k0+4q..+1] and x[token g][k0+4q+2..+3], the same
+// physical columns under the same logical names. A dot product does not
+// depend on the order of its terms' indices, so the MMA computes W x exactly
+// as a sum over the step's 16 columns (fp32 accumulation). The multiply-adds
+// are far below the tensor pipe's rate; the weight stream still bounds the
+// layer, which is why the legacy warp-level instruction suffices here.
+SFC_DEV void mma_16x8x16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+SFC_DEV uint2 ld_stream_v2(const void* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+
+// Shared memory: x_r [tokens][kdim] | parts [per][ks][16 rows][8 tokens] fp32 |
+// own [per][2 vectors][8 tokens] (packed bf16) | counters [per]. A CTA owns
+// the 16-row tiles [t0, t0 + per) of its rank; LL vector u * hidden / 8 + v
+// carries rows 8v .. 8v+7 of token u.
+constexpr int kMmaSteps = 16;  // k-steps whose loads are issued before their MMAs (256 B a thread)
+template <int NR>
+__global__ void __launch_bounds__(kLinearThreads, 2) linear_mma_kernel(const __grid_constant__ LinearParams p) {
+  extern __shared__ __align__(16) unsigned char sm[];
+  const int r = blockIdx.x / p.G;
+  const int kb = blockIdx.x - r * p.G;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+  const uint64_t kdim = p.kdim, nvec = p.hidden / 8, ntiles = p.hidden / 16, steps = kdim / 16;
+  const uint32_t per = p.per_cta, ks = p.ks, tokens = p.tokens;
+  const uint32_t epoch = p.epoch_dev != nullptr ? device_epoch(p.epoch_dev) : p.epoch;
+  if (epoch == 0 || epoch == 0xFFFFFFFFu) {  // device epochs ran out: sfc_reset first
+    if (threadIdx.x == 0) {
+      if (atomicCAS(p.view.status, 0, static_cast<int>(SFC_ERR_EPOCH)) == 0) atomicExch(p.view.status + 1, 0);
+      atomicExch(p.view.status + 2, 1);
+    }
+    return;
+  }
+  const uint64_t t0 = static_cast<uint64_t>(kb) * per;
+  const uint64_t t1 = t0 + per < ntiles ? t0 + per : ntiles;
+  const uint32_t owned = t0 < t1 ? static_cast<uint32_t>(t1 - t0) : 0u;
+
+  uint16_t* xs = reinterpret_cast<uint16_t*>(sm);
+  float* parts = reinterpret_cast<float*>(sm + ((tokens * kdim * 2 + 15) & ~15ull));
+  uint4* ownv = reinterpret_cast<uint4*>(parts + static_cast<uint64_t>(per) * ks * 128);
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(ownv + static_cast<uint64_t>(per) * 16);
+
+  for (uint64_t i = threadIdx.x; i < tokens * kdim / 8; i += blockDim.x) {
+    const uint64_t u = i / (kdim / 8), c = i - u * (kdim / 8);
+    reinterpret_cast<uint4*>(xs)[i] = ld_nc_v4(p.x[r] + u * kdim + c * 8);
+  }
+  for (uint32_t i = threadIdx.x; i < per; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();
+
+  const uint32_t groups = kLinearWarps / ks, grp = warp / ks, h = warp % ks;
+  const uint64_t s_lo = steps * h / ks, s_hi = steps * (h + 1) / ks;  // this warp's k-steps
+  const uint16_t* W = p.W[r];
+  const bool tok_ok = static_cast<uint32_t>(g) < tokens;
+  const uint16_t* xrow = xs + (tok_ok ? g : 0) * kdim + 4 * q;
+  for (uint32_t t = grp; t < owned; t += groups) {
+    const uint16_t* wg = W + ((t0 + t) * 16 + g) * kdim + 4 * q;  // row g; row g + 8 is 8 kdim further
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    uint64_t s = s_lo;
+    for (; s + kMmaSteps <= s_hi; s += kMmaSteps) {
+      uint2 a[kMmaSteps], b[kMmaSteps];
+#pragma unroll
+      for (int i = 0; i < kMmaSteps; ++i) {
+        a[i] = ld_stream_v2(wg + (s + i) * 16);
+        b[i] = ld_stream_v2(wg + 8 * kdim + (s + i) * 16);
+      }
+#pragma unroll
+      for (int i = 0; i < kMmaSteps; ++i) {
+        const uint2 xv = tok_ok ? *reinterpret_cast<const uint2*>(xrow + (s + i) * 16) : make_uint2(0, 0);
+        mma_16x8x16(d, a[i].x, b[i].x, a[i].y, b[i].y, xv.x, xv.y);
+      }
+    }
+    for (; s < s_hi; ++s) {
+      const uint2 a = ld_stream_v2(wg + s * 16), b = ld_stream_v2(wg + 8 * kdim + s * 16);
+      const uint2 xv = tok_ok ? *reinterpret_cast<const uint2*>(xrow + s * 16) : make_uint2(0, 0);
+      mma_16x8x16(d, a.x, b.x, a.y, b.y, xv.x, xv.y);
+    }
+    // d0, d1: row g, tokens 2q, 2q+1; d2, d3: row g + 8, same tokens
+    float* pt = parts + (static_cast<uint64_t>(t) * ks + h) * 128;
+    pt[g * 8 + 2 * q] = d[0];
+    pt[g * 8 + 2 * q + 1] = d[1];
+    pt[(g + 8) * 8 + 2 * q] = d[2];
+    pt[(g + 8) * 8 + 2 * q + 1] = d[3];
+    __threadfence_block();
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) last = atomicAdd(&cnt[t], 1u) == ks - 1;
+    if (__shfl_sync(kFull, last, 0)) {
+      // the last of the tile's ks warps: lane 2u + half builds and pushes
+      // token u's vector of rows 8 half .. 8 half + 7
+      __threadfence_block();
+      const uint32_t u = lane >> 1, half = lane & 1;
+      if (u < tokens) {
+        const volatile float* pv = parts + static_cast<uint64_t>(t) * ks * 128;
+        float y[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const uint32_t row = half * 8 + m;
+          y[m] = pv[row * 8 + u];
+          for (uint32_t j = 1; j < ks; ++j) y[m] += pv[j * 128 + row * 8 + u];
+        }
+        const uint4 own = make_uint4(pack_rn(y[0], y[1]), pack_rn(y[2], y[3]), pack_rn(y[4], y[5]),
+                                     pack_rn(y[6], y[7]));
+        ownv[t * 16 + half * 8 + u] = own;
+        sfc_device::ll_push(p.view, r, epoch, u * nvec + (t0 + t) * 2 + half, own);
+      }
+    }
+  }
+  __syncthreads();  // every vector of the CTA is pushed and its own part stored
+  const uint32_t work = owned * 2 * tokens;
+  for (uint32_t base = 0; base < work; base += kLinearThreads) {
+    const uint32_t i = base + threadIdx.x;
+    const bool act = i < work;
+    // i = (u * owned + t) * 2 + half
+    const uint32_t half = i & 1, ut = i >> 1;
+    const uint32_t u = act ? ut / owned : 0, t = act ? ut - u * owned : 0;
+    const uint64_t v = (t0 + t) * 2 + half;
+    const uint4 own = act ? ownv[t * 16 + half * 8 + u] : make_uint4(0, 0, 0, 0);
+    uint4 out;
+    if (!sfc_device::ll_allreduce_lane<NR>(p.view, r, epoch, u * nvec + v, act, own, &out)) return;
+    if (act) *reinterpret_cast<uint4*>(p.y[r] + u * p.hidden + v * 8) = out;
+  }
+  if (p.epoch_dev != nullptr && lane == 0)
+    finish_device_epoch(p.epoch_dev, p.done_ctr, gridDim.x * (blockDim.x >> 5), epoch + 1);
+}
+
 template <int NR>
 struct LinearRow {
   static const void* get(uint32_t T) {
     switch (T) {
+      case 0: return reinterpret_cast<const void*>(&linear_mma_kernel<NR>);  // tensor-core tile
       case 1: return reinterpret_cast<const void*>(&linear_allreduce_kernel<NR, 1>);
       case 2: return reinterpret_cast<const void*>(&linear_allreduce_kernel<NR, 2>);
       case 4: return reinterpret_cast<const void*>(&linear_allreduce_kernel<NR, 4>);

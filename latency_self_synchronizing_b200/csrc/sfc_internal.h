@@ -126,6 +126,12 @@ inline uint32_t linear_token_tile(uint32_t tokens) { return tokens <= 1 ? 1 : to
 inline size_t linear_smem_bytes(uint64_t kdim, uint32_t T, uint32_t ks, uint32_t per_cta) {
   return kdim * 2 * T + 32ull * ks * T * per_cta + 16ull * T * per_cta + 4ull * per_cta;
 }
+// tensor-core kernel (2..8 tokens, 16-row tiles): x, per-part sums of 16 x 8,
+// own vectors (2 x 8 per tile), counters
+inline size_t linear_mma_smem_bytes(uint64_t kdim, uint32_t tokens, uint32_t ks, uint32_t per_tiles) {
+  return ((tokens * kdim * 2 + 15) & ~15ull) + 512ull * ks * per_tiles + 256ull * per_tiles + 4ull * per_tiles;
+}
+// token_tile 1, 2, 4, 8: the CUDA-core kernel; 0: the tensor-core kernel
 const void* linear_kernel_for(int nranks, uint32_t token_tile);
 
 // Kernel entry for (nranks, protocol, op); null if not provided.

@@ -46,7 +46,7 @@ struct sfc_ctx {
   int occupancy[kNumProtocols][2][2] = {};  // blocks per SM, per (protocol, op, CTA size), 0 = unknown
   int forced_protocol = 0;                // SFC_PROTOCOL: what AUTO resolves to (0 = the selector)
   int smem_optin = 0;                     // opt-in shared memory per block (bytes)
-  int linear_occ[4] = {};                 // fused-linear CTAs per SM per token tile 1/2/4/8 (0 = not queried)
+  int linear_occ[5] = {};                 // fused-linear CTAs per SM: token tile 1/2/4/8, tensor-core (0 = not queried)
 
   // staging for the host-buffer entry point, and the copy streams and
   // events that overlap its copies with the chain segments
@@ -767,8 +767,13 @@ sfc_status sfc_linear_allreduce_tokens(sfc_ctx* c, const void* const* W, const v
                                        size_t hidden, size_t kdim, uint32_t tokens, uint32_t epoch, void* stream) {
   if (c == nullptr || W == nullptr || x == nullptr || y == nullptr) return SFC_ERR_INVALID;
   if (tokens < 1 || tokens > sfc::kLinearMaxTokens) return SFC_ERR_INVALID;
-  const uint32_t T = sfc::linear_token_tile(tokens);
-  if (hidden == 0 || hidden % 8 || hidden * tokens > c->max_count || kdim == 0 || kdim % 8 || kdim * T > 49152)
+  // 3+ tokens on 16-aligned shapes run on the tensor cores (16-row x 8-token
+  // tiles); 1-2 tokens, or ragged shapes, on the CUDA cores (token tile T),
+  // which measured faster there
+  const bool mma = tokens >= 3 && hidden % 16 == 0 && kdim % 16 == 0;
+  const uint32_t T = mma ? 0 : sfc::linear_token_tile(tokens);
+  if (hidden == 0 || hidden % 8 || hidden * tokens > c->max_count || kdim == 0 || kdim % 8 ||
+      kdim * (mma ? tokens : T) > 49152)
     return SFC_ERR_INVALID;
   if (c->region[kLL] == nullptr) return SFC_ERR_UNSUPPORTED;
   if (c->poisoned) return SFC_ERR_ABORTED;
@@ -791,12 +796,13 @@ sfc_status sfc_linear_allreduce_tokens(sfc_ctx* c, const void* const* W, const v
           (a < b && overlap(y[a], yb, y[b], yb)))
         return SFC_ERR_INVALID;
   const void* fn = linear_kernel_for(N, T);
-  // as many CTAs per rank as fit (two per SM), each rank's output vectors
-  // split evenly over its CTAs; ks warps share a vector when that evens out
-  // the 8 warps' work (every part keeps at least 128 column chunks, four per
-  // lane)
-  const uint64_t nvec = hidden / 8, kvec = kdim / 8;
-  const int ti = T == 1 ? 0 : T == 2 ? 1 : T == 4 ? 2 : 3;
+  // as many CTAs per rank as fit (two per SM), each rank's output units
+  // (8-row vectors, or 16-row tiles on the tensor cores) split evenly over
+  // its CTAs; ks warps share a unit when that evens out the 8 warps' work
+  // (every part keeps at least 1024 columns)
+  const uint64_t units = mma ? hidden / 16 : hidden / 8;  // 16-row tiles or 8-row vectors
+  const uint64_t kparts = mma ? kdim / 16 / 64 : kdim / 8 / 128;  // most column parts a unit may split into
+  const int ti = mma ? 4 : T == 1 ? 0 : T == 2 ? 1 : T == 4 ? 2 : 3;
   int occ = c->linear_occ[ti];
   if (occ == 0) {
     if (!cuda_ok(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, c->smem_optin)))
@@ -809,10 +815,10 @@ sfc_status sfc_linear_allreduce_tokens(sfc_ctx* c, const void* const* W, const v
   uint32_t per = 0, ks = 1;
   for (;; --G) {
     if (G < 1) return SFC_ERR_RESOURCES;
-    per = static_cast<uint32_t>((nvec + G - 1) / G);
+    per = static_cast<uint32_t>((units + G - 1) / G);
     double best = -1.0;
     for (uint32_t cand = 1; cand <= 8; cand *= 2) {
-      if (cand > 1 && kvec / cand < 128) break;
+      if (cand > 1 && kparts < cand) break;
       const uint32_t groups = 8 / cand, rounds = (per + groups - 1) / groups;
       const double eff = static_cast<double>(per) / (static_cast<double>(rounds) * groups);
       if (eff > best + 1e-9) {
@@ -821,12 +827,14 @@ sfc_status sfc_linear_allreduce_tokens(sfc_ctx* c, const void* const* W, const v
       }
     }
     // both CTAs of an SM must fit: fewer, larger CTAs if not
-    const size_t smem = sfc::linear_smem_bytes(kdim, T, ks, per);
+    const size_t smem =
+        mma ? sfc::linear_mma_smem_bytes(kdim, tokens, ks, per) : sfc::linear_smem_bytes(kdim, T, ks, per);
     if (smem <= static_cast<size_t>(c->smem_optin) &&
         (G * N <= c->sm_count || 2 * (smem + 1024) <= static_cast<size_t>(c->smem_optin) + 1024))
       break;
   }
-  const int smem = static_cast<int>(sfc::linear_smem_bytes(kdim, T, ks, per));
+  const int smem = static_cast<int>(mma ? sfc::linear_mma_smem_bytes(kdim, tokens, ks, per)
+                                         : sfc::linear_smem_bytes(kdim, T, ks, per));
   p.per_cta = per;
   p.ks = ks;
   p.hidden = hidden;

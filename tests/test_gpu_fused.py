@@ -85,11 +85,13 @@ def test_linear_allreduce_shares_the_epoch_sequence():
         comm.close()
 
 
-# several decode tokens in one pass over the weights (token tiles 2, 4, 8;
-# 3, 5, 6, 7 tokens run in the next tile with the extra tokens masked)
+# several decode tokens in one pass over the weights: 1-2 tokens (and ragged
+# shapes) on the CUDA cores with token tiles 2, 4, 8 (extra tokens masked),
+# 3-8 tokens on 16-aligned shapes on the tensor cores (16 x 8 tiles)
 @pytest.mark.parametrize("n,hidden,kdim,tokens", [(2, 64, 512, 2), (4, 8192, 3584, 4), (8, 1024, 1024, 8),
                                                   (3, 2056, 136, 3), (4, 512, 4096, 5), (2, 1000, 2048, 7),
-                                                  (8, 64, 8, 6), (5, 8192, 1024, 8)])
+                                                  (8, 64, 8, 6), (5, 8192, 1024, 8), (3, 2064, 144, 3),
+                                                  (4, 4096, 2048, 2)])
 def test_linear_allreduce_tokens_within_bound(n, hidden, kdim, tokens):
     w, _ = _case(n, hidden, kdim, seed=hidden * 3 + kdim + n + tokens)
     x = make_inputs(seed=hidden + tokens, k_ops=1, nranks=n, count=tokens * kdim, dist="normal",
