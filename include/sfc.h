@@ -340,12 +340,11 @@ sfc_status sfc_linear_allreduce(sfc_ctx* ctx, const void* const* W, const void* 
  * [tokens][kdim], y[r] bf16 [tokens][hidden]; the weights stream once for
  * all tokens and the all-reduce covers tokens * hidden elements (one epoch).
  * tokens * hidden <= max count of the context; kdim * T <= 49152, T = tokens
- * rounded up to 1, 2, 4 or 8 (3+ tokens on 16-aligned shapes use tensor
- * cores instead, with the x bound tokens * kdim <= 49152).
+ * rounded up to 1, 2, 4 or 8; 2+ tokens with hidden % 16 == 0 and
+ * kdim % 32 == 0 run on the tensor cores instead, with tokens * kdim <= 49152.
  * sfc_linear_allreduce is tokens = 1. Measured on B200 against a library
- * tensor-core GEMM + all-reduce: faster at 1 token, equal at 2, 1.2-1.45x
- * slower at 4-8 tokens (the fused kernel's weight reads are 32-byte pieces of
- * 16 rows at a time there). */
+ * tensor-core GEMM + all-reduce: 1.07-1.13x faster at 1-4 tokens, equal to
+ * 1.13x faster at 8. */
 sfc_status sfc_linear_allreduce_tokens(sfc_ctx* ctx, const void* const* W, const void* const* x, void* const* y,
                                        size_t hidden, size_t kdim, uint32_t tokens, uint32_t epoch, void* stream);
 

@@ -189,18 +189,19 @@ __global__ void __launch_bounds__(kLinearThreads, T >= 8 ? 1 : 2)
 }
 
 // ---------------------------------------------------------------------------
-// 3..8 tokens on the tensor cores (mma.sync m16n8k16, bf16 in, fp32 out).
+// 2..8 tokens on the tensor cores (mma.sync m16n8k16, bf16 in, fp32 out).
 // The tile is 16 rows of W_r (two LL vectors) by 8 token columns (tokens past
-// p.tokens are zero). The k order inside one MMA step is a permutation both
-// operands share, chosen so that every thread reads its weights as two
-// coalesced 8-byte pieces: thread (group g, quad q) takes W[row0 + g][k0 + 4q
-// .. 4q+3] and W[row0 + g + 8][same]; its A registers are (row g, k0+4q..+1),
-// (row g+8, k0+4q..+1), (row g, k0+4q+2..+3), (row g+8, k0+4q+2..+3), which
-// the instruction reads as the logical columns 2q, 2q+1 / 2q+8, 2q+9; its B
-// registers are x[token g][k0+4q..+1] and x[token g][k0+4q+2..+3], the same
-// physical columns under the same logical names. A dot product does not
-// depend on the order of its terms' indices, so the MMA computes W x exactly
-// as a sum over the step's 16 columns (fp32 accumulation). The multiply-adds
+// p.tokens are zero). Columns go in blocks of 32, two MMA steps each, whose
+// k order is a permutation both operands share, chosen so that every thread
+// reads its weights as two 16-byte pieces: thread (group g, quad q) takes
+// W[row0 + g][k0 + 8q .. 8q+7] and W[row0 + g + 8][same]. For the first MMA
+// its A registers are (row g, k0+8q..+1), (row g+8, k0+8q..+1), (row g,
+// k0+8q+2..+3), (row g+8, k0+8q+2..+3), which the instruction reads as the
+// logical columns 2q, 2q+1 / 2q+8, 2q+9; the second MMA takes k0+8q+4..+7 the
+// same way. Its B registers are x[token g] at the same physical columns under
+// the same logical names. A dot product does not depend on the order of its
+// terms' indices, so the MMAs compute W x exactly as a sum over the block's
+// 32 columns (fp32 accumulation). The multiply-adds
 // are far below the tensor pipe's rate; the weight stream still bounds the
 // layer, which is why the legacy warp-level instruction suffices here.
 SFC_DEV void mma_16x8x16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
@@ -222,14 +223,14 @@ SFC_DEV uint2 ld_stream_v2(const void* p) {
 // own [per][2 vectors][8 tokens] (packed bf16) | counters [per]. A CTA owns
 // the 16-row tiles [t0, t0 + per) of its rank; LL vector u * hidden / 8 + v
 // carries rows 8v .. 8v+7 of token u.
-constexpr int kMmaSteps = 16;  // k-steps whose loads are issued before their MMAs (256 B a thread)
+constexpr int kMmaPairs = 8;  // 32-column blocks whose loads are issued before their MMAs (256 B a thread)
 template <int NR>
 __global__ void __launch_bounds__(kLinearThreads, 2) linear_mma_kernel(const __grid_constant__ LinearParams p) {
   extern __shared__ __align__(16) unsigned char sm[];
   const int r = blockIdx.x / p.G;
   const int kb = blockIdx.x - r * p.G;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-  const uint64_t kdim = p.kdim, nvec = p.hidden / 8, ntiles = p.hidden / 16, steps = kdim / 16;
+  const uint64_t kdim = p.kdim, nvec = p.hidden / 8, ntiles = p.hidden / 16, pairs = kdim / 32;
   const uint32_t per = p.per_cta, ks = p.ks, tokens = p.tokens;
   const uint32_t epoch = p.epoch_dev != nullptr ? device_epoch(p.epoch_dev) : p.epoch;
   if (epoch == 0 || epoch == 0xFFFFFFFFu) {  // device epochs ran out: sfc_reset first
@@ -256,31 +257,33 @@ __global__ void __launch_bounds__(kLinearThreads, 2) linear_mma_kernel(const __g
   __syncthreads();
 
   const uint32_t groups = kLinearWarps / ks, grp = warp / ks, h = warp % ks;
-  const uint64_t s_lo = steps * h / ks, s_hi = steps * (h + 1) / ks;  // this warp's k-steps
+  const uint64_t s_lo = pairs * h / ks, s_hi = pairs * (h + 1) / ks;  // this warp's 32-column blocks
   const uint16_t* W = p.W[r];
   const bool tok_ok = static_cast<uint32_t>(g) < tokens;
-  const uint16_t* xrow = xs + (tok_ok ? g : 0) * kdim + 4 * q;
+  const uint16_t* xrow = xs + (tok_ok ? g : 0) * kdim + 8 * q;
   for (uint32_t t = grp; t < owned; t += groups) {
-    const uint16_t* wg = W + ((t0 + t) * 16 + g) * kdim + 4 * q;  // row g; row g + 8 is 8 kdim further
+    const uint16_t* wg = W + ((t0 + t) * 16 + g) * kdim + 8 * q;  // row g; row g + 8 is 8 kdim further
     float d[4] = {0.f, 0.f, 0.f, 0.f};
     uint64_t s = s_lo;
-    for (; s + kMmaSteps <= s_hi; s += kMmaSteps) {
-      uint2 a[kMmaSteps], b[kMmaSteps];
+    for (; s + kMmaPairs <= s_hi; s += kMmaPairs) {
+      uint4 a[kMmaPairs], b[kMmaPairs];
 #pragma unroll
-      for (int i = 0; i < kMmaSteps; ++i) {
-        a[i] = ld_stream_v2(wg + (s + i) * 16);
-        b[i] = ld_stream_v2(wg + 8 * kdim + (s + i) * 16);
+      for (int i = 0; i < kMmaPairs; ++i) {
+        a[i] = ld_stream_v4(wg + (s + i) * 32);
+        b[i] = ld_stream_v4(wg + 8 * kdim + (s + i) * 32);
       }
 #pragma unroll
-      for (int i = 0; i < kMmaSteps; ++i) {
-        const uint2 xv = tok_ok ? *reinterpret_cast<const uint2*>(xrow + (s + i) * 16) : make_uint2(0, 0);
+      for (int i = 0; i < kMmaPairs; ++i) {
+        const uint4 xv = tok_ok ? *reinterpret_cast<const uint4*>(xrow + (s + i) * 32) : make_uint4(0, 0, 0, 0);
         mma_16x8x16(d, a[i].x, b[i].x, a[i].y, b[i].y, xv.x, xv.y);
+        mma_16x8x16(d, a[i].z, b[i].z, a[i].w, b[i].w, xv.z, xv.w);
       }
     }
     for (; s < s_hi; ++s) {
-      const uint2 a = ld_stream_v2(wg + s * 16), b = ld_stream_v2(wg + 8 * kdim + s * 16);
-      const uint2 xv = tok_ok ? *reinterpret_cast<const uint2*>(xrow + s * 16) : make_uint2(0, 0);
+      const uint4 a = ld_stream_v4(wg + s * 32), b = ld_stream_v4(wg + 8 * kdim + s * 32);
+      const uint4 xv = tok_ok ? *reinterpret_cast<const uint4*>(xrow + s * 32) : make_uint4(0, 0, 0, 0);
       mma_16x8x16(d, a.x, b.x, a.y, b.y, xv.x, xv.y);
+      mma_16x8x16(d, a.z, b.z, a.w, b.w, xv.z, xv.w);
     }
     // d0, d1: row g, tokens 2q, 2q+1; d2, d3: row g + 8, same tokens
     float* pt = parts + (static_cast<uint64_t>(t) * ks + h) * 128;

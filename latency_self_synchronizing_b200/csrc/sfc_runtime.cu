@@ -767,10 +767,10 @@ sfc_status sfc_linear_allreduce_tokens(sfc_ctx* c, const void* const* W, const v
                                        size_t hidden, size_t kdim, uint32_t tokens, uint32_t epoch, void* stream) {
   if (c == nullptr || W == nullptr || x == nullptr || y == nullptr) return SFC_ERR_INVALID;
   if (tokens < 1 || tokens > sfc::kLinearMaxTokens) return SFC_ERR_INVALID;
-  // 3+ tokens on 16-aligned shapes run on the tensor cores (16-row x 8-token
-  // tiles); 1-2 tokens, or ragged shapes, on the CUDA cores (token tile T),
-  // which measured faster there
-  const bool mma = tokens >= 3 && hidden % 16 == 0 && kdim % 16 == 0;
+  // 2+ tokens on shapes of whole 16-row, 32-column tiles run on the tensor
+  // cores (16-row x 8-token tiles); one token, or other shapes, on the CUDA
+  // cores (token tile T)
+  const bool mma = tokens >= 2 && hidden % 16 == 0 && kdim % 32 == 0;
   const uint32_t T = mma ? 0 : sfc::linear_token_tile(tokens);
   if (hidden == 0 || hidden % 8 || hidden * tokens > c->max_count || kdim == 0 || kdim % 8 ||
       kdim * (mma ? tokens : T) > 49152)
@@ -801,7 +801,7 @@ sfc_status sfc_linear_allreduce_tokens(sfc_ctx* c, const void* const* W, const v
   // its CTAs; ks warps share a unit when that evens out the 8 warps' work
   // (every part keeps at least 1024 columns)
   const uint64_t units = mma ? hidden / 16 : hidden / 8;  // 16-row tiles or 8-row vectors
-  const uint64_t kparts = mma ? kdim / 16 / 64 : kdim / 8 / 128;  // most column parts a unit may split into
+  const uint64_t kparts = kdim / 1024;  // most column parts a unit may split into
   const int ti = mma ? 4 : T == 1 ? 0 : T == 2 ? 1 : T == 4 ? 2 : 3;
   int occ = c->linear_occ[ti];
   if (occ == 0) {

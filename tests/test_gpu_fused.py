@@ -91,7 +91,7 @@ def test_linear_allreduce_shares_the_epoch_sequence():
 @pytest.mark.parametrize("n,hidden,kdim,tokens", [(2, 64, 512, 2), (4, 8192, 3584, 4), (8, 1024, 1024, 8),
                                                   (3, 2056, 136, 3), (4, 512, 4096, 5), (2, 1000, 2048, 7),
                                                   (8, 64, 8, 6), (5, 8192, 1024, 8), (3, 2064, 144, 3),
-                                                  (4, 4096, 2048, 2)])
+                                                  (4, 4096, 2048, 2), (3, 2064, 160, 3), (2, 1000, 512, 2)])
 def test_linear_allreduce_tokens_within_bound(n, hidden, kdim, tokens):
     w, _ = _case(n, hidden, kdim, seed=hidden * 3 + kdim + n + tokens)
     x = make_inputs(seed=hidden + tokens, k_ops=1, nranks=n, count=tokens * kdim, dist="normal",
