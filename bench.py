@@ -144,6 +144,28 @@ def time_oracle(sample_ops=3, tokens=1, budget_s=25.0):
     return dt / done * 1e6, desc
 
 
+def time_threaded(tokens=TOKENS):
+    """The concurrent CPU model (one thread per rank, C11 atomics, same
+    protocol and chain) on the bench's workload; returns ({tokens: us per
+    all-reduce}, threads, description). Every output is checked against the
+    closed form on op 0 and the last op."""
+    from latency_self_synchronizing_b200.inputs import make_inputs
+    from oracle import reference, threaded
+
+    per = {}
+    for t in tokens:
+        x = make_inputs(seed=0, k_ops=K_OPS, nranks=NRANKS, count=HIDDEN * t, dist="normal", params=(1.0,))
+        out, secs = threaded.chain(PROTOCOL, x)
+        for k in (0, K_OPS - 1):
+            if not all(np.array_equal(out[k, r], reference.allreduce(x[k])) for r in range(NRANKS)):
+                raise RuntimeError("threaded CPU model disagrees with the closed form")
+        per[t] = secs / K_OPS * 1e6
+    threads = NRANKS
+    desc = (f"threaded C model ({PROTOCOL}), {NRANKS} threads, {K_OPS} chained all-reduces per size, "
+            f"hidden {HIDDEN} x {list(tokens)} token(s)")
+    return per, threads, desc
+
+
 def run_reference(args):
     ws, rank, _ = _dist()
     if rank != 0:
@@ -372,10 +394,14 @@ def run_gpu(args):
             "algorithmic_bytes_per_launch": dom["algorithmic_bytes_per_op"] * K_OPS,
             "peak_source": peaks["source"], "kernel": key}
 
-    cpu = None
+    cpu = cpu_threaded = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         v, desc = time_oracle(sample_ops=8)
         cpu = {"value": v, "unit": "us", "cores": 1, "kind": "oracle", "sample": desc}
+        per, threads, desc = time_threaded()
+        cpu_threaded = {"value": per[TOKENS[0]], "unit": "us", "cores": min(threads, os.cpu_count() or 1),
+                        "kind": "concurrent CPU model", "sample": desc,
+                        "us_per_op_by_tokens": {str(t): v for t, v in per.items()}}
 
     if rank == 0:
         line = {
@@ -394,6 +420,7 @@ def run_gpu(args):
                       "headline_ratio": value / (floor["flag_rtt_ns_p50"] / 1e3)},
             "roofline": roof,
             "cpu_baseline": cpu,
+            "cpu_threaded": cpu_threaded,
             "e2e": {"value": e2e_us, "unit": "us", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h2d,
                     "min_max": [min(e2e_ms) * 1e3 / K_OPS, max(e2e_ms) * 1e3 / K_OPS],
                     "what": f"sfc_allreduce_chain_host, {K_OPS} ops at {2 * t1['count']} B/rank, per op"},

@@ -39,6 +39,12 @@ Parity status of each part (what pins it, independent of the code itself):
                      N=2-3, an exhaustive interleaving search at N=2, random and
                      adversarial schedules, and planted mistakes that the checks
                      must catch.
+* ``threaded``    -- (``threaded.c``, plain C, one POSIX thread per rank, C11
+                     atomics) the same protocols on real threads: pinned to the
+                     closed forms under the CPU's own interleavings and seeded
+                     start skews, with planted mistakes (a dropped sentinel
+                     reset, a reversed reduction order) that the checks catch.
+                     Not imported here: it compiles on first use.
 * ``sol``         -- pinned: the worked example on the first page.
 * ``selector``    -- parity unpinned: the pages give no cost-model numbers, so
                      which protocol wins where cannot be checked against them;
