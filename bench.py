@@ -22,6 +22,7 @@ import argparse
 import json
 import os
 import statistics
+import subprocess
 import sys
 import time
 
@@ -398,10 +399,13 @@ def run_gpu(args):
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         v, desc = time_oracle(sample_ops=8)
         cpu = {"value": v, "unit": "us", "cores": 1, "kind": "oracle", "sample": desc}
-        per, threads, desc = time_threaded()
-        cpu_threaded = {"value": per[TOKENS[0]], "unit": "us", "cores": min(threads, os.cpu_count() or 1),
-                        "kind": "concurrent CPU model", "sample": desc,
-                        "us_per_op_by_tokens": {str(t): v for t, v in per.items()}}
+        try:
+            per, threads, desc = time_threaded()
+            cpu_threaded = {"value": per[TOKENS[0]], "unit": "us", "cores": min(threads, os.cpu_count() or 1),
+                            "kind": "concurrent CPU model", "sample": desc,
+                            "us_per_op_by_tokens": {str(t): v for t, v in per.items()}}
+        except (OSError, RuntimeError, subprocess.CalledProcessError) as exc:  # a side figure: keep the line
+            cpu_threaded = {"value": None, "error": f"{type(exc).__name__}: {exc}"}
 
     if rank == 0:
         line = {
