@@ -40,11 +40,13 @@ Parity status of each part (what pins it, independent of the code itself):
                      adversarial schedules, and planted mistakes that the checks
                      must catch.
 * ``threaded``    -- (``threaded.c``, plain C, one POSIX thread per rank, C11
-                     atomics) the same protocols on real threads: pinned to the
+                     atomics) every protocol on real threads: pinned to the
                      closed forms under the CPU's own interleavings and seeded
-                     start skews, with planted mistakes (a dropped sentinel
-                     reset, a reversed reduction order) that the checks catch.
-                     Not imported here: it compiles on first use.
+                     delays, with planted mistakes (a dropped sentinel reset,
+                     a reversed reduction order, one receive buffer, no bottom
+                     barrier, one input buffer in the dual-buffered oneshot)
+                     that the checks catch. Not imported here: it compiles on
+                     first use.
 * ``sol``         -- pinned: the worked example on the first page.
 * ``selector``    -- parity unpinned: the pages give no cost-model numbers, so
                      which protocol wins where cannot be checked against them;

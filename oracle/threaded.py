@@ -22,13 +22,17 @@ import tempfile
 
 import numpy as np
 
-__all__ = ["PROTOCOLS", "build", "chain", "ThreadedError"]
+__all__ = ["PROTOCOLS", "ALLGATHER_PROTOCOLS", "ARGTYPES", "build", "chain", "ThreadedError"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "threaded.c")
 _OUT = os.path.join(_HERE, "_build", "libsfo_threaded.so")
 
-PROTOCOLS = {"ll": 1, "ll128": 2, "sentinel": 3, "barrier_oneshot": 4}
+PROTOCOLS = {"ll": 1, "ll128": 2, "sentinel": 3, "barrier_oneshot": 4, "barrier_twoshot": 5,
+             "barrier_oneshot_db": 6, "ll_twoshot": 7, "sentinel_twoshot": 8}
+ALLGATHER_PROTOCOLS = ("ll", "ll128", "sentinel")
+ARGTYPES = [C.c_int, C.c_int, C.c_int, C.c_size_t, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
+            C.c_double, C.c_int, C.POINTER(C.c_double)]
 _OPS = {"allreduce": 0, "allgather": 1}
 _ERRORS = {1: "invalid arguments", 2: "a wait ran out", 3: "slots not left as the protocol requires",
            4: "out of memory", 5: "thread creation failed"}
@@ -60,18 +64,18 @@ def _load():
     if _lib is None:
         lib = C.CDLL(build())
         lib.sfo_threaded_chain.restype = C.c_int
-        lib.sfo_threaded_chain.argtypes = [C.c_int, C.c_int, C.c_int, C.c_size_t, C.c_int, C.c_void_p,
-                                           C.c_void_p, C.c_void_p, C.c_double, C.c_int,
-                                           C.POINTER(C.c_double)]
+        lib.sfo_threaded_chain.argtypes = ARGTYPES
         _lib = lib
     return _lib
 
 
-def chain(protocol, x, op="allreduce", skew_ns=None, timeout_s=10.0):
+def chain(protocol, x, op="allreduce", skew_ns=None, skew_after=False, timeout_s=10.0):
     """Run len(x) chained operations (epochs 1..k) on x.shape[1] threads.
 
     x: uint16 bf16 bits [k, N, count]. skew_ns: optional uint32 [k, N], a
-    delay before each rank's push. Returns (out, seconds): out is
+    delay of each rank in each operation: before it starts the operation, or
+    with ``skew_after`` between its pushes (or its top barrier) and its
+    first read, a late reader. Returns (out, seconds): out is
     [k, N, count] (all-reduce) or [k, N, N * count] (all-gather); seconds is
     the wall time of the whole chain."""
     x = np.ascontiguousarray(x, dtype=np.uint16)
@@ -86,7 +90,7 @@ def chain(protocol, x, op="allreduce", skew_ns=None, timeout_s=10.0):
     yield_polls = int(n > (os.cpu_count() or 1))
     rc = _load().sfo_threaded_chain(PROTOCOLS[protocol], _OPS[op], n, count, k, x.ctypes.data,
                                     out.ctypes.data, None if skew is None else skew.ctypes.data,
-                                    float(timeout_s), yield_polls, C.byref(secs))
+                                    int(bool(skew_after)), float(timeout_s), yield_polls, C.byref(secs))
     if rc != 0:
         raise ThreadedError(rc)
     return out, secs.value
