@@ -217,21 +217,30 @@ class Communicator:
         """outputs[r] = inputs[0] || ... || inputs[N-1]."""
         self._one(self._lib.sfc_allgather, Op.ALLGATHER, inputs, outputs, protocol, epoch, stream)
 
+    def _device_tensor(self, t, dtypes, min_numel, exact, what):
+        """Checks a tensor the kernel reads or writes directly: on this
+        communicator's device (a host pointer would be dereferenced by the
+        GPU), contiguous, of one of `dtypes`, with enough entries."""
+        ok = (isinstance(t, torch.Tensor) and t.is_cuda and t.device.index == self._device and t.dtype in dtypes
+              and t.is_contiguous() and (t.numel() == min_numel if exact else t.numel() >= min_numel))
+        if not ok:
+            raise ValueError(f"{what} must be a contiguous {'/'.join(str(d) for d in dtypes)} tensor on cuda:"
+                             f"{self._device} with {'' if exact else 'at least '}{min_numel} entries")
+        return C.c_void_p(t.data_ptr())
+
+    def _timings_ptr(self, timings, k_ops):
+        if timings is None:
+            return None
+        return self._device_tensor(timings, (torch.int64,), k_ops + 1, False, "timings")
+
     def _chain(self, fn, in_table, out_table, count, k_ops, protocol, epoch, skew_ns, timings, stream):
         n = self.nranks
         for name, t in (("in_table", in_table), ("out_table", out_table)):
-            if t.dtype != torch.int64 or not t.is_cuda or t.numel() != k_ops * n:
-                raise ValueError(f"{name} must be an int64 CUDA tensor of {k_ops * n} pointers")
+            self._device_tensor(t, (torch.int64,), k_ops * n, True, name)
         skew_p = None
         if skew_ns is not None:
-            if skew_ns.dtype not in (torch.int32, torch.uint32) or skew_ns.numel() != k_ops * n:
-                raise ValueError("skew_ns must be an int32 CUDA tensor of k_ops * N entries")
-            skew_p = C.c_void_p(skew_ns.data_ptr())
-        tim_p = None
-        if timings is not None:
-            if timings.dtype != torch.int64 or timings.numel() < k_ops + 1:
-                raise ValueError("timings must be an int64 CUDA tensor of k_ops + 1 entries")
-            tim_p = C.c_void_p(timings.data_ptr())
+            skew_p = self._device_tensor(skew_ns, (torch.int32, torch.uint32), k_ops * n, True, "skew_ns")
+        tim_p = self._timings_ptr(timings, k_ops)
         e = 0 if epoch is None else int(epoch)  # 0 = the next epoch
         _check(fn(self._ctx, int(k_ops), C.c_void_p(in_table.data_ptr()), C.c_void_p(out_table.data_ptr()),
                   int(count), 0, int(as_protocol(protocol)), e, skew_p, tim_p, _stream_handle(stream)),
@@ -256,7 +265,7 @@ class Communicator:
         k, n, count = in_host.shape
         if n != self.nranks or tuple(out_host.shape) != (k, n, count):
             raise ValueError("shape mismatch")
-        tim_p = None if timings is None else C.c_void_p(timings.data_ptr())
+        tim_p = self._timings_ptr(timings, k)
         e = 0 if epoch is None else int(epoch)  # 0 = the next epoch
         _check(self._lib.sfc_allreduce_chain_host(self._ctx, int(k), C.c_void_p(in_host.data_ptr()),
                                                   C.c_void_p(out_host.data_ptr()), int(count), 0,

@@ -182,3 +182,49 @@ def _struct_fields(name):
 def test_binding_structs_match_the_header(cname, pyname):
     py = [f[0] for f in getattr(_lib, pyname)._fields_]
     assert _struct_fields(cname) == py
+
+
+def _bare_communicator(n=2):
+    """A Communicator with no context behind it: enough to reach the
+    argument checks that run before any library call."""
+    from latency_self_synchronizing_b200 import api
+
+    class NoCalls:
+        def __getattr__(self, name):
+            def call(*args):
+                raise AssertionError(f"{name} reached the library")
+            call.__name__ = name
+            return call
+
+    c = api.Communicator.__new__(api.Communicator)
+    c.nranks, c._device, c._ctx, c._lib = n, 0, None, NoCalls()
+    return c
+
+
+def test_chain_rejects_host_tensors_the_kernel_would_dereference():
+    """Pointer tables, skews and timing buffers are read or written by the
+    GPU itself: host tensors are refused before anything is launched."""
+    import torch
+
+    c = _bare_communicator(2)
+    table = torch.zeros(2 * 3, dtype=torch.int64)  # host memory
+    with pytest.raises(ValueError, match="in_table"):
+        c.allreduce_chain(table, table, 8, 3, protocol="ll")
+    with pytest.raises(ValueError, match="timings"):
+        c._timings_ptr(torch.zeros(4, dtype=torch.int64), 3)
+    with pytest.raises(ValueError, match="skew_ns"):
+        c._device_tensor(torch.zeros(6, dtype=torch.int32), (torch.int32,), 6, True, "skew_ns")
+    assert c._timings_ptr(None, 3) is None
+
+
+def test_host_chain_rejects_bad_host_operands():
+    import torch
+
+    c = _bare_communicator(2)
+    good = torch.zeros(3, 2, 8, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="in_host"):
+        c.allreduce_chain_host(torch.zeros(3, 2, 8, dtype=torch.float32), good)
+    with pytest.raises(ValueError, match="shape"):
+        c.allreduce_chain_host(good, torch.zeros(3, 2, 9, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="timings"):
+        c.allreduce_chain_host(good, good.clone(), timings=torch.zeros(4, dtype=torch.int64))
