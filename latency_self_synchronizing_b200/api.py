@@ -191,12 +191,15 @@ class Communicator:
         want_out = count if op == Op.ALLREDUCE else n * count
         ins, outs = self._ptrs_in, self._ptrs_out
         bf16 = torch.bfloat16
+        dev = self._device
         for r in range(n):
             a, b = inputs[r], outputs[r]
             if not (a.is_cuda and b.is_cuda and a.dtype is bf16 and b.dtype is bf16 and a.is_contiguous()
                     and b.is_contiguous()):
                 _dev_ptr(a, "input")
                 _dev_ptr(b, "output")
+            if a.get_device() != dev or b.get_device() != dev:
+                raise ValueError(f"operands must be on cuda:{dev}, the communicator's device")
             if a.numel() != count:
                 raise ValueError("all inputs must have the same number of elements")
             if b.numel() != want_out:
@@ -285,6 +288,8 @@ class Communicator:
         for w, x_, y_ in zip(weights, xs, ys):
             if tuple(w.shape) != (hidden, kdim) or x_.numel() != tokens * kdim or y_.numel() != tokens * hidden:
                 raise ValueError("shape mismatch")
+        if any(t.get_device() != self._device for t in (*weights, *xs, *ys)):
+            raise ValueError(f"operands must be on cuda:{self._device}, the communicator's device")
         W = (C.c_void_p * n)(*[_dev_ptr(w, "weight") for w in weights])
         X = (C.c_void_p * n)(*[_dev_ptr(t, "input") for t in xs])
         Y = (C.c_void_p * n)(*[_dev_ptr(t, "output") for t in ys])

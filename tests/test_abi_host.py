@@ -228,3 +228,16 @@ def test_host_chain_rejects_bad_host_operands():
         c.allreduce_chain_host(good, torch.zeros(3, 2, 9, dtype=torch.bfloat16))
     with pytest.raises(ValueError, match="timings"):
         c.allreduce_chain_host(good, good.clone(), timings=torch.zeros(4, dtype=torch.int64))
+
+
+def test_single_ops_and_linear_reject_host_operands():
+    import torch
+
+    c = _bare_communicator(2)
+    x = [torch.zeros(8, dtype=torch.bfloat16) for _ in range(2)]
+    with pytest.raises(TypeError, match="CUDA"):
+        c.allreduce(x, [t.clone() for t in x], protocol="ll")
+    w = [torch.zeros(16, 8, dtype=torch.bfloat16) for _ in range(2)]
+    y = [torch.zeros(16, dtype=torch.bfloat16) for _ in range(2)]
+    with pytest.raises(ValueError, match="cuda:0"):
+        c.linear_allreduce(w, x, y)
