@@ -205,3 +205,26 @@ def test_selfsync_twoshot_survives_a_single_buffer(tmp_path, proto):
     for after in (0, 1):
         rc, out = _run(lib, proto, x, _late_last_rank(8, 4, 500_000), after=after)
         assert rc in (0, 3) and _matches(out, x)
+
+
+def _golden_cases():
+    path = os.path.join(os.path.dirname(__file__), "golden", "rank_order_sum.txt")
+    for line in open(path):
+        line = line.split("#")[0].strip()
+        if line:
+            left, right = line.split("->")
+            parts = left.split()
+            n = int(parts[1])
+            yield parts[0], [int(h, 16) for h in parts[2:2 + n]], int(right.split("|")[0], 16)
+
+
+@pytest.mark.parametrize("proto", PROTOS)
+def test_hand_derived_order_sensitive_cases(proto):
+    """The hand-derived cases whose answer depends on the rank order give
+    the derived bits on real threads too, whatever order the units land."""
+    for name, xs, want in _golden_cases():
+        n, count = len(xs), 97
+        x = np.empty((6, n, count), dtype=np.uint16)
+        x[:] = np.array(xs, dtype=np.uint16)[None, :, None]
+        out, _ = threaded.chain(proto, x)
+        assert np.all(out == want), (name, proto)
