@@ -1,0 +1,32 @@
+"""bench.py measures the named decode workload it reports (no GPU needed)."""
+import importlib.util
+import os
+
+from latency_self_synchronizing_b200.workloads import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_bench_constants_are_the_decode_h8192_workload():
+    b = _bench()
+    w = WORKLOADS["decode_h8192"]
+    assert b.NRANKS == w["nranks"]
+    assert [b.PROTOCOL] == w["protocols"]
+    assert [b.HIDDEN * t for t in b.TOKENS] == w["counts"]
+    assert b.K_OPS == w["k_ops"]
+    cfg = b._config()
+    assert cfg["workload"] == "decode_h8192"
+    assert cfg["bytes_per_rank"] == [2 * c for c in w["counts"]]
+    assert cfg["nranks"] == w["nranks"] and cfg["protocol"] == b.PROTOCOL and cfg["k_ops_per_chain"] == b.K_OPS
+
+
+def test_bench_metric_is_time_like():
+    b = _bench()
+    assert "p50" in b.METRIC
