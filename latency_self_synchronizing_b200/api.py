@@ -107,9 +107,12 @@ def _dev_ptr(t, name):
 
 
 def pointer_table(rows):
-    """[[tensor per rank] per operation] -> int64 CUDA tensor of data pointers."""
+    """[[tensor per rank] per operation] -> int64 CUDA tensor of data pointers
+    (every operand on one device, the table on that device too)."""
     ptrs = [_dev_ptr(t, "chain operand") for row in rows for t in row]
     dev = rows[0][0].device
+    if any(t.device != dev for row in rows for t in row):
+        raise ValueError(f"every chain operand must be on {dev}")
     return torch.tensor(ptrs, dtype=torch.int64, device=dev)
 
 

@@ -242,3 +242,12 @@ def test_single_ops_and_linear_reject_host_operands():
     y = [torch.zeros(16, dtype=torch.bfloat16) for _ in range(2)]
     with pytest.raises(ValueError, match="cuda:0"):
         c.linear_allreduce(w, x, y)
+
+
+def test_pointer_table_refuses_host_tensors():
+    import torch
+
+    from latency_self_synchronizing_b200 import api
+
+    with pytest.raises(TypeError, match="CUDA"):
+        api.pointer_table([[torch.zeros(8, dtype=torch.bfloat16)]])
