@@ -167,6 +167,22 @@ def time_threaded(tokens=TOKENS):
     return per, threads, desc
 
 
+def cpu_baselines(sample_ops=8, tokens=TOKENS):
+    """The bench line's two CPU figures: the oracle's simulator on a bounded
+    sample (`cpu_baseline`) and the concurrent C model on whole chains
+    (`cpu_threaded`, reported as an error string if it cannot run)."""
+    v, desc = time_oracle(sample_ops=sample_ops)
+    cpu = {"value": v, "unit": "us", "cores": 1, "kind": "oracle", "sample": desc, "host_cores": os.cpu_count()}
+    try:
+        per, threads, desc = time_threaded(tokens)
+        cpu_threaded = {"value": per[tokens[0]], "unit": "us", "cores": min(threads, os.cpu_count() or 1),
+                        "kind": "concurrent CPU model", "sample": desc, "host_cores": os.cpu_count(),
+                        "us_per_op_by_tokens": {str(t): v for t, v in per.items()}}
+    except (OSError, RuntimeError, subprocess.CalledProcessError) as exc:  # a side figure: keep the line
+        cpu_threaded = {"value": None, "error": f"{type(exc).__name__}: {exc}"}
+    return cpu, cpu_threaded
+
+
 def run_reference(args):
     ws, rank, _ = _dist()
     if rank != 0:
@@ -184,7 +200,8 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": value / 1e3, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": _config(),
-        "cpu_baseline": {"value": value, "unit": "us", "cores": 1, "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "us", "cores": 1, "kind": "oracle", "sample": desc,
+                         "host_cores": os.cpu_count()},
         "e2e": {"value": value, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -397,15 +414,7 @@ def run_gpu(args):
 
     cpu = cpu_threaded = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        v, desc = time_oracle(sample_ops=8)
-        cpu = {"value": v, "unit": "us", "cores": 1, "kind": "oracle", "sample": desc}
-        try:
-            per, threads, desc = time_threaded()
-            cpu_threaded = {"value": per[TOKENS[0]], "unit": "us", "cores": min(threads, os.cpu_count() or 1),
-                            "kind": "concurrent CPU model", "sample": desc,
-                            "us_per_op_by_tokens": {str(t): v for t, v in per.items()}}
-        except (OSError, RuntimeError, subprocess.CalledProcessError) as exc:  # a side figure: keep the line
-            cpu_threaded = {"value": None, "error": f"{type(exc).__name__}: {exc}"}
+        cpu, cpu_threaded = cpu_baselines()
 
     if rank == 0:
         line = {

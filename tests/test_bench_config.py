@@ -30,3 +30,14 @@ def test_bench_constants_are_the_decode_h8192_workload():
 def test_bench_metric_is_time_like():
     b = _bench()
     assert "p50" in b.METRIC
+
+
+def test_cpu_baselines_shape():
+    """The two CPU figures of the bench line, on the smallest sample."""
+    import json
+
+    b = _bench()
+    cpu, thr = b.cpu_baselines(sample_ops=1, tokens=(1,))
+    assert cpu["kind"] == "oracle" and cpu["cores"] == 1 and cpu["value"] > 0 and cpu["host_cores"] >= 1
+    assert thr["value"] > 0 and thr["cores"] >= 1 and set(thr["us_per_op_by_tokens"]) == {"1"}
+    json.dumps({"cpu_baseline": cpu, "cpu_threaded": thr})
