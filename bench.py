@@ -408,7 +408,8 @@ def run_gpu(args):
     ach = dom["achieved_gbs_launch"]
     key = f"sfc_kernel<{NRANKS}, sentinel, allreduce> x {K_OPS} ops, {dom['bytes_per_rank']} B/rank"
     roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": ach / peaks["hbm_gbs"], "traffic": recorded_traffic(key),
+            "frac": ach / peaks["hbm_gbs"],
+            "traffic": recorded_traffic(key, grid=NRANKS * dom["launch_shape"][0], block=dom["launch_shape"][1]),
             "algorithmic_bytes_per_launch": dom["algorithmic_bytes_per_op"] * K_OPS,
             "peak_source": peaks["source"], "kernel": key}
 
@@ -449,29 +450,30 @@ def run_gpu(args):
     return 0
 
 
+KERNEL_SOURCES = ("latency_self_synchronizing_b200/csrc/sfc_kernels.cu",
+                  "latency_self_synchronizing_b200/csrc/sfc_device.cuh",
+                  "latency_self_synchronizing_b200/csrc/sfc_internal.h",
+                  "include/sfc.h", "include/sfc_ll_device.cuh")
+
+
 def kernel_sources_sha():
-    """SHA-256 over the sources that decide what the chain kernels do and how
-    they are launched (kernels, device helpers, internal header, runtime); the
-    selector's measured table, the floor benchmark, the allocation-free
-    entry point and the fused linear kernel do not change a chain launch and
-    are left out."""
+    """SHA-256 over the sources of the chain kernels' device code (kernels,
+    device helpers, the parameter block and its constants, the public
+    headers they include). How a chain is launched is checked live instead:
+    a recorded capture also names its grid and block."""
     import hashlib
 
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "latency_self_synchronizing_b200", "csrc")
-    skip = ("sfc_cost_table.h", "sfc_floor.cu", "sfc_noalloc.cu", "sfc_fused.cu")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")) and name not in skip:
-            h.update(name.encode())
-            h.update(open(os.path.join(csrc, name), "rb").read())
-    h.update(open(os.path.join(ROOT, "include", "sfc.h"), "rb").read())
+    for rel in KERNEL_SOURCES:
+        h.update(rel.encode())
+        h.update(open(os.path.join(ROOT, rel), "rb").read())
     return h.hexdigest()
 
 
-def recorded_traffic(key):
+def recorded_traffic(key, grid=None, block=None):
     """DRAM bytes per launch recorded from an ncu capture of this kernel and
     workload (profiles/ncu_traffic.json), or None when the kernel sources have
-    changed since the capture."""
+    changed since the capture or the launch now has another grid or block."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         rec = json.load(open(path))
@@ -480,7 +482,11 @@ def recorded_traffic(key):
     if rec.get("kernel_sources_sha") != kernel_sources_sha():
         return None
     ent = rec.get("launches", {}).get(key)
-    return None if ent is None else float(ent["dram_bytes_per_launch"])
+    if ent is None:
+        return None
+    if (grid is not None and ent.get("grid") != grid) or (block is not None and ent.get("block") != block):
+        return None
+    return float(ent["dram_bytes_per_launch"])
 
 
 def _peaks():

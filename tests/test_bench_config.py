@@ -41,3 +41,20 @@ def test_cpu_baselines_shape():
     assert cpu["kind"] == "oracle" and cpu["cores"] == 1 and cpu["value"] > 0 and cpu["host_cores"] >= 1
     assert thr["value"] > 0 and thr["cores"] >= 1 and set(thr["us_per_op_by_tokens"]) == {"1"}
     json.dumps({"cpu_baseline": cpu, "cpu_threaded": thr})
+
+
+def test_recorded_traffic_is_keyed_on_device_sources_and_launch_shape(monkeypatch):
+    b = _bench()
+    key = "sfc_kernel<4, sentinel, allreduce> x 160 ops, 131072 B/rank"
+    import json
+
+    rec = json.load(open(os.path.join(ROOT, "profiles", "ncu_traffic.json")))
+    ent = rec["launches"][key]
+    if rec["kernel_sources_sha"] == b.kernel_sources_sha():
+        assert b.recorded_traffic(key, grid=ent["grid"], block=ent["block"]) == ent["dram_bytes_per_launch"]
+        assert b.recorded_traffic(key, grid=ent["grid"] // 2, block=ent["block"]) is None
+        assert b.recorded_traffic(key, grid=ent["grid"], block=ent["block"] // 2) is None
+    monkeypatch.setattr(b, "kernel_sources_sha", lambda: "0" * 64)  # the kernels changed since the capture
+    assert b.recorded_traffic(key, grid=ent["grid"], block=ent["block"]) is None
+    for rel in b.KERNEL_SOURCES:
+        assert os.path.exists(os.path.join(ROOT, rel)), rel
