@@ -456,17 +456,43 @@ KERNEL_SOURCES = ("latency_self_synchronizing_b200/csrc/sfc_kernels.cu",
                   "include/sfc.h", "include/sfc_ll_device.cuh")
 
 
+def _code_only(text):
+    """C/C++ source with comments removed and whitespace runs collapsed
+    (string and character literals kept as they are)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        ch = text[i]
+        if text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif ch in "\"'":
+            j = i + 1
+            while j < n and text[j] != ch:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        else:
+            out.append(ch)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_sources_sha():
-    """SHA-256 over the sources of the chain kernels' device code (kernels,
+    """SHA-256 over the code of the chain kernels' device sources (kernels,
     device helpers, the parameter block and its constants, the public
-    headers they include). How a chain is launched is checked live instead:
-    a recorded capture also names its grid and block."""
+    headers they include), comments and layout excluded. How a chain is
+    launched is checked live instead: a recorded capture also names its grid
+    and block."""
     import hashlib
 
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
         h.update(rel.encode())
-        h.update(open(os.path.join(ROOT, rel), "rb").read())
+        h.update(_code_only(open(os.path.join(ROOT, rel), encoding="utf-8").read()).encode())
     return h.hexdigest()
 
 

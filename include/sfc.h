@@ -37,7 +37,9 @@
  *     operation consumes one, and a call must pass exactly the next one
  *     (sfc_next_epoch), else SFC_ERR_EPOCH; 0, never an epoch itself,
  *     stands for the next one. All-reduce and all-gather share the
- *     sequence. Parity = epoch & 1 selects the scratch buffer.
+ *     sequence. Parity = epoch & 1 selects the scratch buffer. Once epoch
+ *     2^32 - 1 has been used the sequence is spent: sfc_next_epoch returns 0
+ *     and every call returns SFC_ERR_EPOCH until sfc_reset.
  *   - Device epochs (sfc_config.device_epochs): the next epoch is a word in
  *     device memory that each launch reads when it starts and that its last
  *     warp advances when every warp has finished, so a call enqueued now

@@ -151,7 +151,9 @@ sfc_status check_common(sfc_ctx* c, sfc_op op, size_t count, sfc_dtype dtype, in
   if (count > c->max_count) return SFC_ERR_INVALID;
   if (c->poisoned) return SFC_ERR_ABORTED;
   if (c->cfg.device_epochs) return first_epoch == 0 ? SFC_OK : SFC_ERR_EPOCH;  // the kernel checks the range
-  if (first_epoch != c->next_epoch) return SFC_ERR_EPOCH;
+  // next_epoch is 0 once epoch 2^32 - 1 has been used: the sequence is spent
+  // (an epoch of 0 would validate against zero-filled flags) until sfc_reset
+  if (first_epoch == 0 || first_epoch != c->next_epoch) return SFC_ERR_EPOCH;
   if (static_cast<uint64_t>(first_epoch) + static_cast<uint64_t>(k_ops) - 1 > 0xFFFFFFFFull) return SFC_ERR_EPOCH;
   return SFC_OK;
 }
@@ -752,7 +754,7 @@ sfc_status sfc_reserve_epochs(sfc_ctx* c, uint32_t k, uint32_t* first) {
   if (c == nullptr || first == nullptr || k == 0) return SFC_ERR_INVALID;
   if (c->cfg.device_epochs) return SFC_ERR_UNSUPPORTED;  // the host does not know the epoch
   if (c->poisoned) return SFC_ERR_ABORTED;
-  if (static_cast<uint64_t>(c->next_epoch) + k - 1 > 0xFFFFFFFFull) return SFC_ERR_EPOCH;
+  if (c->next_epoch == 0 || static_cast<uint64_t>(c->next_epoch) + k - 1 > 0xFFFFFFFFull) return SFC_ERR_EPOCH;
   *first = c->next_epoch;
   c->next_epoch += k;
   return SFC_OK;
@@ -778,7 +780,7 @@ sfc_status sfc_linear_allreduce_tokens(sfc_ctx* c, const void* const* W, const v
   if (c->region[kLL] == nullptr) return SFC_ERR_UNSUPPORTED;
   if (c->poisoned) return SFC_ERR_ABORTED;
   epoch = resolve_epoch(c, epoch);
-  if (c->cfg.device_epochs ? epoch != 0 : epoch != c->next_epoch) return SFC_ERR_EPOCH;
+  if (c->cfg.device_epochs ? epoch != 0 : (epoch == 0 || epoch != c->next_epoch)) return SFC_ERR_EPOCH;
   const int N = c->nranks;
   sfc::LinearParams p{};
   p.epoch_dev = c->cfg.device_epochs ? c->d_epoch : nullptr;

@@ -167,3 +167,37 @@ def test_env_overrides(monkeypatch):
         assert comm.select_protocol("allgather", 2048) != api.Protocol.LL_TWOSHOT
     finally:
         comm.close()
+
+
+def test_spent_epoch_sequence_is_refused_until_reset():
+    """After epoch 2^32 - 1 the host sequence is spent: a wrap to 0 would
+    validate against zero-filled LL flags, so every call is refused with
+    SFC_ERR_EPOCH (nothing launched) until sfc_reset."""
+    comm = api.Communicator(2, 4096)
+    try:
+        x = make_inputs(seed=9, k_ops=2, nranks=2, count=64)
+        ins, outs = _ops(x)
+        assert comm.reserve_epochs(0xFFFFFFFE) == 1  # epochs 1 .. 2^32 - 2, never launched
+        assert comm.next_epoch == 0xFFFFFFFF
+        comm.allreduce(ins.tensors(0), outs.tensors(0), protocol="ll")  # the last epoch
+        torch.cuda.synchronize()
+        assert comm.status()[0] == api.Status.OK
+        np.testing.assert_array_equal(outs.bits()[0, 0], reference.allreduce(x[0]))
+        assert comm.next_epoch == 0
+        launches = comm.launch_count
+        for proto in ("ll", "sentinel", "barrier_oneshot"):
+            with pytest.raises(api.SfcError) as ei:
+                comm.allreduce(ins.tensors(1), outs.tensors(1), protocol=proto)
+            assert ei.value.status == api.Status.EPOCH
+        with pytest.raises(api.SfcError) as ei:
+            comm.reserve_epochs(1)
+        assert ei.value.status == api.Status.EPOCH
+        assert comm.launch_count == launches
+        comm.reset()
+        assert comm.next_epoch == 1
+        comm.allreduce(ins.tensors(1), outs.tensors(1), protocol="ll")
+        torch.cuda.synchronize()
+        assert comm.status()[0] == api.Status.OK
+        np.testing.assert_array_equal(outs.bits()[1, 1], reference.allreduce(x[1]))
+    finally:
+        comm.close()
