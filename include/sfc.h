@@ -345,7 +345,7 @@ sfc_status sfc_linear_allreduce(sfc_ctx* ctx, const void* const* W, const void* 
  * rounded up to 1, 2, 4 or 8; 2+ tokens with hidden % 16 == 0 and
  * kdim % 32 == 0 run on the tensor cores instead, with tokens * kdim <= 49152.
  * sfc_linear_allreduce is tokens = 1. Measured on B200 against a library
- * tensor-core GEMM + all-reduce: 1.07-1.13x faster at 1-4 tokens, equal to
+ * tensor-core GEMM + all-reduce: 1.07-1.16x faster at 1-4 tokens, equal to
  * 1.13x faster at 8. */
 sfc_status sfc_linear_allreduce_tokens(sfc_ctx* ctx, const void* const* W, const void* const* x, void* const* y,
                                        size_t hidden, size_t kdim, uint32_t tokens, uint32_t epoch, void* stream);
