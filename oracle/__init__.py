@@ -47,6 +47,12 @@ Parity status of each part (what pins it, independent of the code itself):
                      barrier, one input buffer in the dual-buffered oneshot)
                      that the checks catch. Not imported here: it compiles on
                      first use.
+* ``linear``      -- the row-parallel linear layer and its all-reduce (the
+                     fused layer): pinned by hand-worked values, one-hot
+                     inputs that pick weight columns, additivity over ranks
+                     and tokens, and an error bound that must cover simulated
+                     fp32 / bf16 arithmetic in four summation orders while
+                     catching a dropped block of products.
 * ``sol``         -- pinned: the worked example on the first page.
 * ``selector``    -- parity unpinned: the pages give no cost-model numbers, so
                      which protocol wins where cannot be checked against them;
@@ -54,4 +60,4 @@ Parity status of each part (what pins it, independent of the code itself):
                      examples.
 """
 
-from . import bf16, reference, protocols, simulator, exhaustive, sol, selector  # noqa: F401
+from . import bf16, reference, protocols, simulator, exhaustive, sol, selector, linear  # noqa: F401
