@@ -216,6 +216,95 @@ def _config():
             "parallelism": "replicas (emulated ranks inside each GPU)"}
 
 
+# ---------------------------------------------------------------- targets
+TARGET_RANKS = (2, 4, 8)
+TARGET_SMALL = (1024, 16384)        # bytes per rank: latency target, <= 3x the flag round trip
+TARGET_LARGE = (1 << 20, 16 << 20)  # bytes per rank: bandwidth target, >= 0.5 of the HBM roofline
+L2_BYTES = 126 * 1024 * 1024
+
+
+def large_point_inputs(nranks, nbytes, l2_bytes=L2_BYTES):
+    """Distinct inputs per chain for a bandwidth point: enough operations
+    that the chain's inputs are at least twice the L2 (every operation reads
+    its inputs from HBM), at least 8, at most 128 and at most 1.5 GB."""
+    per_op = nranks * nbytes
+    need = -(-2 * l2_bytes // per_op)
+    cap = max(8, (3 << 29) // per_op)
+    return int(min(128, cap, max(8, need)))
+
+
+def measure_targets(dev, floor_us, peak_gbs, large_only=False):
+    """The selector's protocol at the target points, measured as chains
+    outside the timed region: p50 per operation against the flag round-trip
+    floor at small sizes; algorithmic and recorded-DRAM bandwidth fractions
+    at large sizes (inputs larger than L2). large_only skips the small
+    points (the launches an ncu traffic capture records, in this order)."""
+    import torch
+
+    from latency_self_synchronizing_b200 import api, sweep
+
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    small, large = [], []
+    for n in TARGET_RANKS:
+        sel = api.Communicator(n, 1 << 10)  # every protocol provisioned: the selector's own choice
+        try:
+            chosen = {b: sel.select_protocol("allreduce", b, n).name.lower() for b in TARGET_SMALL + TARGET_LARGE}
+        finally:
+            sel.close()
+        for b in () if large_only else TARGET_SMALL:
+            proto = chosen[b]
+            comm = api.Communicator(n, b, protocols=[proto])
+            try:
+                pt = sweep.measure_point(comm, "allreduce", proto, b // 2, 100, 3, gen, dev)
+            finally:
+                comm.close()
+            small.append({"nranks": n, "bytes_per_rank": b, "protocol": proto, "p50_us": pt["p50_us"],
+                          "p99_us": pt["p99_us"], "floor_ratio": pt["p50_us"] / floor_us,
+                          "met": pt["p50_us"] / floor_us <= 3.0})
+        for b in TARGET_LARGE:
+            proto = chosen[b]
+            k = large_point_inputs(n, b)
+            comm = api.Communicator(n, b, protocols=[proto])
+            try:
+                pt = sweep.measure_point(comm, "allreduce", proto, b // 2, k, 3, gen, dev, distinct=k)
+                shape = comm.launch_shape("allreduce", proto, b // 2)
+            finally:
+                comm.close()
+                torch.cuda.empty_cache()
+            alg = pt["algorithmic_bytes"] / (pt["p50_us"] * 1e-6) / 1e9
+            key = f"sfc_kernel<{n}, {proto}, allreduce> x {k} ops, {b} B/rank"
+            traffic = recorded_traffic(key, grid=n * shape[0], block=shape[1])
+            dram = None if traffic is None else traffic / k / (pt["p50_us"] * 1e-6) / 1e9
+            large.append({"nranks": n, "bytes_per_rank": b, "protocol": proto, "p50_us": pt["p50_us"],
+                          "p99_us": pt["p99_us"], "k_ops": k, "algorithmic_bytes_per_op": pt["algorithmic_bytes"],
+                          "algorithmic_gbs": alg, "algorithmic_frac": alg / peak_gbs,
+                          "dram_bytes_per_op": None if traffic is None else traffic / k,
+                          "dram_gbs": dram, "dram_frac": None if dram is None else dram / peak_gbs,
+                          "met": alg / peak_gbs >= 0.5, "ncu_key": key})
+    return {"small": small, "large": large,
+            "what": "selector's protocol per point; chains of 100 ops (small, 8 distinct inputs) or of k distinct "
+                    "inputs totalling >= 2x L2 (large); p50 from completion stamps; floor = flag round trip; "
+                    "dram = ncu-recorded DRAM bytes of the same launch (null when the kernels changed since)",
+            "small_met": all(p["met"] for p in small) if small else None,
+            "large_met": all(p["met"] for p in large)}
+
+
+def run_targets_only(args):
+    """--targets-only: the target points alone, one JSON line (no timed step,
+    no floor unless small points are measured)."""
+    import torch
+
+    from latency_self_synchronizing_b200 import api
+
+    torch.cuda.set_device(_dist()[2])
+    dev = torch.device("cuda", _dist()[2])
+    floor_us = float("nan") if args.large_only else api.measure_floor(500)["flag_rtt_ns_p50"] / 1e3
+    t = measure_targets(dev, floor_us, _peaks()["hbm_gbs"], large_only=args.large_only)
+    print(json.dumps({"targets": t, "floor_us": floor_us}))
+    return 0
+
+
 # -------------------------------------------------------------------- GPU
 def run_gpu(args):
     import torch
@@ -232,7 +321,7 @@ def run_gpu(args):
     peaks = _peaks()
     max_count = HIDDEN * max(TOKENS)
     comm = api.Communicator(NRANKS, max_count * 2, protocols=[PROTOCOL, "ll", "ll128"])
-    floor = api.measure_floor(4000)
+    floor = api.measure_floor(500)
 
     # operands: 160 distinct inputs per rank, outputs alternate two buffers
     chains = []
@@ -355,6 +444,19 @@ def run_gpu(args):
     b.record(stream)
     torch.cuda.synchronize()
     single_b2b = a.elapsed_time(b) * 1e3 / n_calls
+    # the same call prepared once (sfc_plan_create), launched back to back
+    plan = comm.plan(xs, ys, protocol=PROTOCOL)
+    for _ in range(20):
+        plan.launch()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n_calls):
+        plan.launch()
+    b.record(stream)
+    torch.cuda.synchronize()
+    plan_b2b = a.elapsed_time(b) * 1e3 / n_calls
+    plan.close()
     iso = []
     for _ in range(50):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -391,10 +493,12 @@ def run_gpu(args):
         raise RuntimeError("graph-replayed all-reduce differs from the eager one")
     del graph
     gcomm.close()
-    single = {"back_to_back_us": single_b2b, "isolated_us_p50": _percentile(iso, 0.5),
+    single = {"back_to_back_us": single_b2b, "plan_back_to_back_us": plan_b2b,
+              "isolated_us_p50": _percentile(iso, 0.5),
               "graph_replay_us": statistics.median(g_us), "unit": "us",
               "what": f"sfc_allreduce, one launch per call, {2 * t1['count']} B/rank; back to back = "
-                      f"{n_calls} calls between two events; isolated = one call between two events; "
+                      f"{n_calls} calls between two events; plan = the same call prepared once "
+                      f"(sfc_plan_create) and launched {n_calls} times; isolated = one call between two events; "
                       f"graph replay = {K_OPS} calls captured in one CUDA graph (device epochs), per call"}
     st, info = comm.status()
     if st != api.Status.OK:
@@ -413,6 +517,8 @@ def run_gpu(args):
             "algorithmic_bytes_per_launch": dom["algorithmic_bytes_per_op"] * K_OPS,
             "peak_source": peaks["source"], "kernel": key}
 
+    targets = None if args.no_targets else measure_targets(dev, floor["flag_rtt_ns_p50"] / 1e3, peaks["hbm_gbs"])
+
     cpu = cpu_threaded = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu, cpu_threaded = cpu_baselines()
@@ -424,15 +530,20 @@ def run_gpu(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": _config(), "per_size": per_size,
             "floor": {"flag_rtt_us_p50": floor["flag_rtt_ns_p50"] / 1e3,
-                      "flag_rtt_us_p99": floor["flag_rtt_ns_p99"] / 1e3,
-                      "flag_rtt_us_fastest_pair": floor["flag_rtt_ns_min_pair"] / 1e3,
-                      "flag_rtt_us_slowest_pair": floor["flag_rtt_ns_max_pair"] / 1e3,
-                      "sm_pairs": floor["pairs"],
+                      "flag_rtt_us_p10": floor["flag_rtt_ns_p10"] / 1e3,
+                      "flag_rtt_us_p90": floor["flag_rtt_ns_p90"] / 1e3,
+                      "flag_rtt_us_fastest_trial": floor["flag_rtt_ns_min_pair"] / 1e3,
+                      "flag_rtt_us_slowest_trial": floor["flag_rtt_ns_max_pair"] / 1e3,
+                      "flag_rtt_us_by_location": [v / 1e3 for v in floor["flag_rtt_ns_by_location"]],
+                      "initiator_sms": floor["initiator_sm"], "responder_sms": floor["responder_sm"],
+                      "trials": floor["pairs"],
+                      "statistic": "median over (SM pair x flag address) trials of each trial's median round trip",
                       "l2_rtt_us": floor["l2_rtt_ns_p50"] / 1e3,
                       "sol_analogue_us": (2 * floor["l2_rtt_ns_p50"] + floor["flag_rtt_ns_p50"] / 2) / 1e3,
                       "globaltimer_step_ns": floor["globaltimer_step_ns"], "sm_clock_ghz": floor["sm_clock_ghz"],
                       "headline_ratio": value / (floor["flag_rtt_ns_p50"] / 1e3)},
             "roofline": roof,
+            "targets": targets,
             "cpu_baseline": cpu,
             "cpu_threaded": cpu_threaded,
             "e2e": {"value": e2e_us, "unit": "us", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h2d,
@@ -481,18 +592,34 @@ def _code_only(text):
     return " ".join("".join(out).split())
 
 
+def _nvcc_version():
+    from latency_self_synchronizing_b200 import build
+
+    try:
+        out = subprocess.run([build._nvcc(), "--version"], capture_output=True, text=True, timeout=60).stdout
+    except (OSError, RuntimeError, subprocess.SubprocessError):
+        return "nvcc: unknown"
+    return " ".join(line for line in out.splitlines() if "release" in line or "Build" in line)
+
+
 def kernel_sources_sha():
     """SHA-256 over the code of the chain kernels' device sources (kernels,
     device helpers, the parameter block and its constants, the public
-    headers they include), comments and layout excluded. How a chain is
-    launched is checked live instead: a recorded capture also names its grid
-    and block."""
+    headers they include), comments and layout excluded, plus the nvcc
+    architecture flags, compile flags and compiler version the library is
+    built with. How a chain is launched is checked live instead: a recorded
+    capture also names its grid and block."""
     import hashlib
+
+    from latency_self_synchronizing_b200 import build
 
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
         h.update(rel.encode())
         h.update(_code_only(open(os.path.join(ROOT, rel), encoding="utf-8").read()).encode())
+    flags = [f for f in build.FLAGS if not f.startswith("/")]  # include paths differ between machines
+    h.update(" ".join(build.ARCH + flags).encode())
+    h.update(_nvcc_version().encode())
     return h.hexdigest()
 
 
@@ -531,9 +658,14 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["sfc", "reference"], default="sfc")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-targets", action="store_true", help="skip the selector target points")
+    ap.add_argument("--targets-only", action="store_true", help="measure only the selector target points")
+    ap.add_argument("--large-only", action="store_true", help="with --targets-only: the >= 1 MB points only")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.targets_only:
+        return run_targets_only(args)
     return run_gpu(args)
 
 

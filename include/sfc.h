@@ -146,17 +146,26 @@ typedef struct {
   sfc_cost_entry c[2][SFC_NUM_PROTOCOLS][SFC_MAX_RANKS + 1]; /* [op][protocol][nranks] */
 } sfc_cost_model;
 
+#define SFC_FLOOR_SMS 8        /* initiator SMs, and as many responder SMs */
+#define SFC_FLOOR_LOCATIONS 8  /* flag addresses (different L2 homes) */
+
 typedef struct {
-  double flag_rtt_ns_p50;   /* two CTAs on different SMs ping-pong a flag; median
-                               over all round trips of 16 SM pairs */
-  double flag_rtt_ns_p99;
-  double flag_rtt_ns_min_pair; /* median of the fastest / slowest SM pair */
+  /* Flag round trip between two CTAs on different SMs, measured for every
+   * (initiator, responder) pair of a fixed SM set chosen by %smid at each of
+   * SFC_FLOOR_LOCATIONS flag addresses: one trial per (pair, location), its
+   * median over the trial's round trips. */
+  double flag_rtt_ns_p50;      /* median over the trials: the floor */
+  double flag_rtt_ns_p10;      /* 10th / 90th percentile over the trials */
+  double flag_rtt_ns_p90;
+  double flag_rtt_ns_min_pair; /* fastest / slowest trial */
   double flag_rtt_ns_max_pair;
-  int pairs;
-  double l2_rtt_ns_p50;     /* dependent L2-hit loads, one thread */
-  double sm_clock_ghz;      /* clock64 ticks per globaltimer ns during the run */
-  double globaltimer_step_ns; /* smallest nonzero globaltimer increment seen */
-  int sm_a, sm_b;           /* SMs the two ping-pong CTAs ran on (last trial) */
+  double flag_rtt_ns_by_location[SFC_FLOOR_LOCATIONS]; /* median over the pairs at each address */
+  int initiator_sm[SFC_FLOOR_SMS]; /* %smid of the initiators and responders */
+  int responder_sm[SFC_FLOOR_SMS];
+  int pairs;                   /* trials: SM pairs x locations */
+  double l2_rtt_ns_p50;        /* dependent L2-hit loads, one thread */
+  double sm_clock_ghz;         /* clock64 ticks per globaltimer ns during the run */
+  double globaltimer_step_ns;  /* smallest nonzero globaltimer increment seen */
 } sfc_floor_result;
 
 /* Create a context for `nranks` (2..8) emulated ranks on the current CUDA
@@ -206,6 +215,24 @@ sfc_status sfc_allreduce_chain(sfc_ctx* ctx, int k_ops, const void* const* in_ta
                                void* const* out_table, size_t count, sfc_dtype dtype,
                                sfc_protocol protocol, uint32_t first_epoch,
                                const uint32_t* skew_ns, uint64_t* timings, void* stream);
+
+/* A prepared single all-reduce or all-gather, for callers that issue one
+ * collective at a time on fixed buffers (a decode step that cannot chain its
+ * layers' all-reduces into one launch). sfc_plan_create does once what every
+ * sfc_allreduce / sfc_allgather call does: the argument and operand checks
+ * (as sfc_allreduce; count == 0 -> SFC_ERR_INVALID), the protocol choice
+ * (SFC_PROTO_AUTO -> the selector), the kernel and the launch shape.
+ * sfc_plan_launch then takes the context's next epoch and launches on
+ * `stream`: per call it costs little more than the CUDA launch. The operand
+ * pointers are fixed at creation (the host arrays are copied); their
+ * contents may change between launches. Launches share the context's epoch
+ * sequence with every other call. A plan is valid while its context lives:
+ * destroy plans first. Not thread-safe with other calls on the context. */
+typedef struct sfc_plan sfc_plan;
+sfc_status sfc_plan_create(sfc_ctx* ctx, sfc_op op, const void* const* in, void* const* out, size_t count,
+                           sfc_dtype dtype, sfc_protocol protocol, sfc_plan** plan);
+sfc_status sfc_plan_launch(sfc_plan* plan, void* stream);
+sfc_status sfc_plan_destroy(sfc_plan* plan);
 
 /* The all-gather counterpart of sfc_allreduce_chain (out entries hold
  * N*count elements). */
@@ -294,7 +321,13 @@ sfc_status sfc_set_silent_rank(sfc_ctx* ctx, int silent_rank);
  * its buffers): a flag round trip between two CTAs on different SMs and the
  * L2 hit latency. The speed-of-light bound of "Why Microseconds Matter in AI
  * Infrastructure", section "Defining the physical lower bound", is built
- * from such round trips. iters >= 16. */
+ * from such round trips. The SM pairs are fixed by %smid (every SM hosts
+ * exactly one CTA of the measuring launch): SFC_FLOOR_SMS initiators and as
+ * many responders spread evenly over the sorted SM ids, every initiator
+ * with every responder, at SFC_FLOOR_LOCATIONS flag addresses, since where
+ * a flag's L2 home sits moves one pair's round trip by up to 0.6 us on B200.
+ * iters (>= 16) round trips per trial; the first iters / 8 (at most 64)
+ * warm the lines and are not counted. */
 sfc_status sfc_measure_floor(int iters, sfc_floor_result* out);
 
 /* Number of kernel launches this context has issued (all entry points). */
@@ -369,16 +402,30 @@ sfc_status sfc_check_guards(sfc_ctx* ctx);
  *   in / out: HOST arrays of `nranks` (2..8) DEVICE pointers, 16-byte
  *   aligned, `count` bf16 elements each, no overlap; result as sfc_allreduce
  *   (rank-order fp32 sum, one bf16 rounding), every rank the same bits.
- *   count > SFC_NOALLOC_MAX_COUNT -> SFC_ERR_INVALID; count == 0 -> no-op.
+ *   count > SFC_NOALLOC_MAX_COUNT -> SFC_ERR_INVALID.
+ * Set-up: the first call on a device (any count, with that device current)
+ * looks up the array's device address (cudaGetSymbolAddress), the SM count
+ * and the kernel's occupancy. That lookup may load this library's device code
+ * and place the array in device memory, so it can fail where memory has run
+ * out: make one call with count == 0 (in, out and nranks are then ignored and
+ * nothing is launched) on every device at start-up, before any stream capture.
  * Each call clears the part of the array it uses (cudaMemsetAsync on
  * `stream`), then launches; it calls no cudaMalloc, cudaFree or allocating
- * library routine. The first call on a device looks up the array's device
- * address (cudaGetSymbolAddress) with that device current: make that first
- * call before any stream capture. All calls share the one array and it keeps
- * the last call's contents, so calls that overlap on the GPU (other streams,
- * other threads) race: order them. Device-side errors are not reported. */
+ * library routine. All calls share the one array and it keeps the last call's
+ * contents, so calls that overlap on the GPU (other streams, other threads)
+ * race: order them.
+ * Errors on the device (a wait that ran out, bounded by SFC_TIMEOUT_MS or
+ * 50 ms) stay recorded in the array: every later call then exits at once
+ * without writing its outputs, until sfc_noalloc_status has read them. */
 sfc_status sfc_allreduce_noalloc(const void* const* in, void* const* out, int nranks, size_t count,
                                  void* stream);
+
+/* Device status of the allocation-free all-reduce on the current device,
+ * read after every earlier call on `stream` (synchronizes the stream):
+ * SFC_OK, or the first error recorded (SFC_ERR_TIMEOUT: *info = the
+ * operation, rank and source of the wait that ran out, as sfc_get_status).
+ * Reading clears it, so later calls run again. Allocates nothing. */
+sfc_status sfc_noalloc_status(void* stream, uint32_t* info);
 
 #ifdef __cplusplus
 }

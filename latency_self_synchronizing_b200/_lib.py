@@ -39,11 +39,17 @@ class LLView(C.Structure):
                 ("status", C.c_void_p), ("timeout_ns", C.c_uint64)]
 
 
+SFC_FLOOR_SMS = 8
+SFC_FLOOR_LOCATIONS = 8
+
+
 class FloorResult(C.Structure):
-    _fields_ = [("flag_rtt_ns_p50", C.c_double), ("flag_rtt_ns_p99", C.c_double),
-                ("flag_rtt_ns_min_pair", C.c_double), ("flag_rtt_ns_max_pair", C.c_double), ("pairs", C.c_int),
-                ("l2_rtt_ns_p50", C.c_double), ("sm_clock_ghz", C.c_double),
-                ("globaltimer_step_ns", C.c_double), ("sm_a", C.c_int), ("sm_b", C.c_int)]
+    _fields_ = [("flag_rtt_ns_p50", C.c_double), ("flag_rtt_ns_p10", C.c_double), ("flag_rtt_ns_p90", C.c_double),
+                ("flag_rtt_ns_min_pair", C.c_double), ("flag_rtt_ns_max_pair", C.c_double),
+                ("flag_rtt_ns_by_location", C.c_double * SFC_FLOOR_LOCATIONS),
+                ("initiator_sm", C.c_int * SFC_FLOOR_SMS), ("responder_sm", C.c_int * SFC_FLOOR_SMS),
+                ("pairs", C.c_int), ("l2_rtt_ns_p50", C.c_double), ("sm_clock_ghz", C.c_double),
+                ("globaltimer_step_ns", C.c_double)]
 
 
 # (name, restype, argtypes) for every entry point of include/sfc.h
@@ -79,7 +85,12 @@ SIGNATURES = [
                                   C.c_uint32, _P]),
     ("sfc_linear_allreduce_tokens", _S, [_P, C.POINTER(_P), C.POINTER(_P), C.POINTER(_P), C.c_size_t, C.c_size_t,
                                           C.c_uint32, C.c_uint32, _P]),
+    ("sfc_plan_create", _S, [_P, C.c_int, C.POINTER(_P), C.POINTER(_P), C.c_size_t, C.c_int, C.c_int,
+                             C.POINTER(_P)]),
+    ("sfc_plan_launch", _S, [_P, _P]),
+    ("sfc_plan_destroy", _S, [_P]),
     ("sfc_allreduce_noalloc", _S, [C.POINTER(_P), C.POINTER(_P), C.c_int, C.c_size_t, _P]),
+    ("sfc_noalloc_status", _S, [_P, C.POINTER(C.c_uint32)]),
 ]
 
 _lib = None

@@ -13,7 +13,7 @@ import torch
 from . import _lib
 
 __all__ = [
-    "Status", "Protocol", "Op", "SfcError", "Communicator", "pointer_table", "measure_floor",
+    "Status", "Protocol", "Op", "SfcError", "Communicator", "Plan", "pointer_table", "measure_floor",
     "algorithmic_bytes", "select_protocol_model", "default_cost_model", "status_string", "cost_estimate",
 ]
 
@@ -141,9 +141,13 @@ class Communicator:
         self._device = torch.cuda.current_device()
         self._ptrs_in = (C.c_void_p * self.nranks)()
         self._ptrs_out = (C.c_void_p * self.nranks)()
+        self._plans = []
 
     # ----------------------------------------------------------- lifecycle
     def close(self):
+        for pl in getattr(self, "_plans", []):
+            pl.close()  # plans go before their context
+        self._plans = []
         if getattr(self, "_ctx", None):
             self._lib.sfc_destroy(self._ctx)
             self._ctx = None
@@ -214,6 +218,29 @@ class Communicator:
         rc = fn(self._ctx, ins, outs, count, 0, proto, e, _stream_handle(stream, self._device))
         if rc != 0:
             raise SfcError(rc, fn.__name__)
+
+    def plan(self, inputs, outputs, op="allreduce", protocol="auto"):
+        """A prepared single collective on fixed operands (sfc_plan_create):
+        its launch() takes the next epoch and launches, nothing else."""
+        n = self.nranks
+        if len(inputs) != n or len(outputs) != n:
+            raise ValueError(f"need {n} inputs and {n} outputs")
+        o = as_op(op)
+        count = inputs[0].numel()
+        want_out = count if o == Op.ALLREDUCE else n * count
+        for a, b in zip(inputs, outputs):
+            _dev_ptr(a, "input")
+            _dev_ptr(b, "output")
+            if a.get_device() != self._device or b.get_device() != self._device:
+                raise ValueError(f"operands must be on cuda:{self._device}, the communicator's device")
+            if a.numel() != count or b.numel() != want_out:
+                raise ValueError("operand sizes differ")
+        ins = (C.c_void_p * n)(*[t.data_ptr() for t in inputs])
+        outs = (C.c_void_p * n)(*[t.data_ptr() for t in outputs])
+        h = C.c_void_p()
+        _check(self._lib.sfc_plan_create(self._ctx, int(o), ins, outs, count, 0, int(as_protocol(protocol)),
+                                         C.byref(h)), "sfc_plan_create")
+        return Plan(self, h, (tuple(inputs), tuple(outputs)))
 
     def allreduce(self, inputs, outputs, protocol="auto", epoch=None, stream=None):
         """outputs[r] = rank-order fp32 sum of inputs, rounded once to bf16."""
@@ -356,7 +383,36 @@ def select_protocol_model(model, op, bytes_per_rank, nranks):
                                                           int(nranks)))
 
 
-def measure_floor(iters=20000):
+class Plan:
+    """A prepared collective of a Communicator (see Communicator.plan). It
+    keeps its operand tensors alive; close() (or the communicator's close)
+    releases it."""
+
+    def __init__(self, comm, handle, keep):
+        self._comm = comm
+        self._h = handle
+        self._keep = keep
+        self._launch = comm._lib.sfc_plan_launch
+        self._dev = comm._device
+        comm._plans.append(self)
+
+    def launch(self, stream=None):
+        rc = self._launch(self._h, _stream_handle(stream, self._dev))
+        if rc != 0:
+            raise SfcError(rc, "sfc_plan_launch")
+
+    def close(self):
+        if self._h is not None and self._h.value:
+            self._comm._lib.sfc_plan_destroy(self._h)
+        self._h = None
+
+
+def measure_floor(iters=500):
+    """sfc_measure_floor as a dict (arrays as lists)."""
     r = _lib.FloorResult()
     _check(_lib.load().sfc_measure_floor(int(iters), C.byref(r)), "sfc_measure_floor")
-    return {f: getattr(r, f) for f, _ in _lib.FloorResult._fields_}
+    out = {}
+    for f, _ in _lib.FloorResult._fields_:
+        v = getattr(r, f)
+        out[f] = list(v) if isinstance(v, C.Array) else v
+    return out

@@ -109,6 +109,14 @@ SFC_DEV uint64_t ld_acq_u64(const void* p) {
   return v;
 }
 SFC_DEV void fence_acq_rel() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+// Release fence: with a later strong write it forms a release pattern (every
+// earlier access of the thread, and those ordered before it by a barrier, is
+// visible to whoever observes that write through an acquire pattern). It
+// waits for the thread's outstanding stores: about 0.5 us on B200.
+SFC_DEV void fence_rel() { asm volatile("fence.release.gpu;" ::: "memory"); }
+// Acquire fence: with an earlier strong read it forms an acquire pattern.
+// It waits for no stores: measured as cheap as no fence on B200.
+SFC_DEV void fence_acq() { asm volatile("fence.acquire.gpu;" ::: "memory"); }
 
 // ---- read-only inputs (never written while a kernel runs) -----------------
 SFC_DEV uint4 ld_nc_v4(const void* p) {

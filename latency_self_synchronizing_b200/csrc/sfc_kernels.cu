@@ -26,7 +26,8 @@
 //  * Sentinel: the reset is the write half of the atomic exchange that reads
 //    the data, so it is ordered with the data by atomicity, not by a fence.
 //  * LL128: the writer's release fence between data and flags also orders
-//    every earlier read of the thread before its next flags.
+//    every earlier access of the thread (its reads of the previous
+//    operation's lines included) before its next flags.
 //
 // Within an operation a warp polls all its sources at once (independent
 // loads, one round trip per poll) and the warp decides with a vote whether
@@ -105,6 +106,9 @@ SFC_DEV bool scratch_in_bounds(const KParams& p, const void* ptr, uint64_t bytes
   } while (0)
 #endif
 
+// Source rank of receive slot j of rank r (slots skip the own rank).
+SFC_DEV int src_rank(int j, int r) { return j < r ? j : j + 1; }
+
 // LL layout shared with the public device API (one definition).
 SFC_DEV uint64_t ll_off(uint64_t v, int half) { return sfc_device::ll_offset(v, half); }
 
@@ -160,7 +164,7 @@ SFC_DEV bool ll_poll(const KParams& p, int r, int op, uint32_t e, uint64_t gtid,
         }
       }
       if (!__any_sync(kFull, need != 0u)) break;
-      if (ww.tick(p, op, r, need ? (__ffs(need) - 1) % (N - 1) : -1)) return false;
+      if (ww.tick(p, op, r, need ? src_rank((__ffs(need) - 1) % (N - 1), r) : -1)) return false;
     }
 #pragma unroll
     for (int i = 0; i < K; ++i) {
@@ -224,7 +228,7 @@ SFC_DEV bool ll_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid, u
 // Sentinel poll + reduce, K vectors at a time, sources indexed j = 0..N-2
 // (as in the LL poll); two bits per (vector, source): its low and high 8-byte
 // unit.
-template <int N, int OP, int K>
+template <int N, int OP, int K, bool kLoadPoll>
 SFC_DEV bool sentinel_poll(const KParams& p, int r, int op, uint64_t gtid, uint64_t gstride, uint8_t* my,
                            const uint16_t* in_r, uint16_t* out_r) {
   constexpr uint64_t kFill = ~0ull;
@@ -253,8 +257,17 @@ SFC_DEV bool sentinel_poll(const KParams& p, int r, int op, uint64_t gtid, uint6
         for (int j = 0; j < N - 1; ++j) {
           const int u = 2 * (i * (N - 1) + j);
           uint8_t* s = my + static_cast<uint64_t>(j) * p.slot_stride + v[i] * 16;
-          if (cur & (1u << u)) SFC_SCRATCH(p, s, 8, a[i][j] = atom_exch_u64(s, kFill));
-          if (cur & (2u << u)) SFC_SCRATCH(p, s + 8, 8, b[i][j] = atom_exch_u64(s + 8, kFill));
+          if (kLoadPoll) {
+            if (cur & (3u << u)) {
+              uint64_t ta = kFill, tb = kFill;
+              SFC_SCRATCH(p, s, 16, ld_rlx_v2u64(s, ta, tb));
+              if (cur & (1u << u)) a[i][j] = ta;
+              if (cur & (2u << u)) b[i][j] = tb;
+            }
+          } else {
+            if (cur & (1u << u)) SFC_SCRATCH(p, s, 8, a[i][j] = atom_exch_u64(s, kFill));
+            if (cur & (2u << u)) SFC_SCRATCH(p, s + 8, 8, b[i][j] = atom_exch_u64(s + 8, kFill));
+          }
         }
       }
 #pragma unroll
@@ -267,7 +280,18 @@ SFC_DEV bool sentinel_poll(const KParams& p, int r, int op, uint64_t gtid, uint6
         }
       }
       if (!__any_sync(kFull, need != 0u)) break;
-      if (ww.tick(p, op, r, need ? ((__ffs(need) - 1) / 2) % (N - 1) : -1)) return false;
+      if (ww.tick(p, op, r, need ? src_rank(((__ffs(need) - 1) / 2) % (N - 1), r) : -1)) return false;
+    }
+    if (kLoadPoll) {  // the vector is taken from every source: write the fill back
+#pragma unroll
+      for (int i = 0; i < K; ++i) {
+        if (v[i] >= nvec) continue;
+#pragma unroll
+        for (int j = 0; j < N - 1; ++j) {
+          uint8_t* s = my + static_cast<uint64_t>(j) * p.slot_stride + v[i] * 16;
+          SFC_SCRATCH(p, s, 16, st_rlx_v2u64(s, kFill, kFill));
+        }
+      }
     }
 #pragma unroll
     for (int i = 0; i < K; ++i) {
@@ -298,10 +322,22 @@ SFC_DEV bool sentinel_poll(const KParams& p, int r, int op, uint64_t gtid, uint6
 // Raw data into a slot pre-filled with 0xFFFF. The writer moves each 8 bytes
 // as one single-copy-atomic .b64 element, so an 8-byte unit of the slot is
 // either all fill or all data, and data never equals the fill (inputs never
-// hold 0xFFFF elements). The reader polls each 8-byte unit with an atomic
-// exchange against the fill: a result other than the fill is the data, and
-// the same atomic operation has already written the fill back (the reset).
-template <int N, int OP>
+// hold 0xFFFF elements). Two ways to take and reset the units:
+//  * exchange (kLoadPoll = false, small messages): the reader polls each
+//    8-byte unit with an atomic exchange against the fill: a result other
+//    than the fill is the data, and the same atomic operation has already
+//    written the fill back (the reset). One L2 atomic per unit and per poll
+//    that still finds the fill; lowest latency.
+//  * load + store (kLoadPoll = true, large messages): the reader polls with
+//    16-byte relaxed loads, writes the fill back with a relaxed store once a
+//    vector is complete, and ends the operation with an acquire fence and a
+//    release fence. A writer reuses the slot two epochs later only after it
+//    has seen this rank's next push (its poll followed by its own acquire
+//    fence), so the release / acquire pair orders the resets before that
+//    reuse. No atomics: at (N - 1) x bytes >= 448 KB the L2's atomic
+//    throughput, not the round trip, bounds the exchange polls, and the
+//    release fence (about 0.5 us) costs less than the atomics it saves.
+template <int N, int OP, bool kLoadPoll>
 SFC_DEV bool sentinel_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid, uint64_t gstride,
                          const Operands& io) {
   const uint64_t count = p.count;
@@ -329,7 +365,13 @@ SFC_DEV bool sentinel_op(const KParams& p, int r, int op, uint32_t e, uint64_t g
   prefetch_next_input(io.in_next, gtid, gstride, nvec);
 
   uint8_t* my = slot_ptr<N>(p, r, par, r == 0 ? 1 : 0);
-  return sentinel_poll<N, OP, 1>(p, r, op, gtid, gstride, my, in_r, out_r);
+  if (!kLoadPoll) return sentinel_poll<N, OP, 1, false>(p, r, op, gtid, gstride, my, in_r, out_r);
+  const bool ok = sentinel_poll<N, OP, 1, true>(p, r, op, gtid, gstride, my, in_r, out_r);
+  // acquire (after this operation's polls) + release (before the next
+  // operation's pushes): a peer that sees the next push has seen the resets
+  fence_acq();
+  fence_rel();
+  return ok;
 }
 
 // =================================================================== LL128
@@ -337,10 +379,14 @@ SFC_DEV bool sentinel_op(const KParams& p, int r, int op, uint32_t e, uint64_t g
 // lines: lane l serves line 4g + (l >> 3), sub-slot s = l & 7; lanes s < 7
 // carry 16 data bytes at line offset 16 s, lane 7 carries the last 8 data
 // bytes (offset 112) and the flag (offset 120). Writers store all data,
-// __syncwarp + fence.acq_rel.gpu, then the flags (release pattern); readers
-// poll flags with relaxed loads, fence.acq_rel.gpu + __syncwarp (acquire
-// pattern), then load the data. Flags of up to B line groups are polled at
-// once.
+// __syncwarp + fence.release.gpu, then the flags (release pattern: the warp
+// barrier orders the other lanes' data stores before the flag lane's fence);
+// readers poll flags with relaxed loads, fence.acquire.gpu + __syncwarp
+// (acquire pattern, handed to the other lanes by the barrier), then load the
+// data. The acquire fence waits for no store and costs next to nothing on
+// B200; the release fence waits for the data stores to complete, which is
+// the one round trip LL128 pays that LL does not. Flags of up to B line
+// groups are polled at once.
 template <int N>
 struct LL128Batch {
   static constexpr int B = N >= 16 ? 1 : 16 / N;  // B * N <= 16 flags in flight per lane
@@ -381,7 +427,7 @@ SFC_DEV bool ll128_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid
       }
     }
     __syncwarp();
-    fence_acq_rel();
+    fence_rel();
     for (uint64_t g = wg; g < ngroups; g += wstride) {
       const uint64_t L = g * kLL128LinesPerWarp + lsel;
       if (L < nlines && sub == 7) {
@@ -438,7 +484,7 @@ SFC_DEV bool ll128_op(const KParams& p, int r, int op, uint32_t e, uint64_t gtid
       if (!__any_sync(kFull, need != 0u)) break;
       if (ww.tick(p, op, r, -1)) return false;
     }
-    fence_acq_rel();
+    fence_acq();
     __syncwarp();
 #pragma unroll 1
     for (int b = 0; b < B; ++b) {
@@ -555,7 +601,7 @@ SFC_DEV bool poll_vecs(const KParams& p, uint8_t* base, uint64_t v, uint32_t e, 
       }
     }
     if (!__any_sync(kFull, pend != 0u)) break;
-    if (ww.tick(p, op, r, pend ? __ffs(pend) - 1 : -1)) return false;
+    if (ww.tick(p, op, r, pend ? (kLLenc ? __ffs(pend) - 1 : (__ffs(pend) - 1) / 2) : -1)) return false;
   }
 #pragma unroll
   for (int q = 0; q < N; ++q) {
@@ -940,7 +986,9 @@ __global__ void __launch_bounds__(kThreads, MinBlocks<N, PROTO>::value) sfc_kern
     if (PROTO == kLL)
       ok = ll_op<N, OP>(p, r, op, e, gtid, gstride, io);
     else if (PROTO == kSentinel)
-      ok = sentinel_op<N, OP>(p, r, op, e, gtid, gstride, io);
+      ok = sentinel_op<N, OP, false>(p, r, op, e, gtid, gstride, io);
+    else if (PROTO == kSentinelLoadPoll)
+      ok = sentinel_op<N, OP, true>(p, r, op, e, gtid, gstride, io);
     else if (PROTO == kLL128)
       ok = ll128_op<N, OP>(p, r, op, e, gtid, gstride, io);
     else if (PROTO == kLL128Fast)
@@ -990,10 +1038,15 @@ struct Row {
     t[N][kLL128Fast][kAllreduce] = reinterpret_cast<const void*>(&sfc_kernel<N, kLL128Fast, kAllreduce>);
     t[N][kLL128Fast][kAllgather] = reinterpret_cast<const void*>(&sfc_kernel<N, kLL128Fast, kAllgather>);
   }
+  static void fill_load_poll(const void* (&t)[kMaxRanks + 1][2]) {
+    t[N][kAllreduce] = reinterpret_cast<const void*>(&sfc_kernel<N, kSentinelLoadPoll, kAllreduce>);
+    t[N][kAllgather] = reinterpret_cast<const void*>(&sfc_kernel<N, kSentinelLoadPoll, kAllgather>);
+  }
 };
 
 struct Table {
   const void* t[kMaxRanks + 1][kNumProtocols][2] = {};
+  const void* load_poll[kMaxRanks + 1][2] = {};  // the sentinel's large-message kernels
   Table() {
     Row<2>::fill(t);
     Row<3>::fill(t);
@@ -1002,15 +1055,32 @@ struct Table {
     Row<6>::fill(t);
     Row<7>::fill(t);
     Row<8>::fill(t);
+    Row<2>::fill_load_poll(load_poll);
+    Row<3>::fill_load_poll(load_poll);
+    Row<4>::fill_load_poll(load_poll);
+    Row<5>::fill_load_poll(load_poll);
+    Row<6>::fill_load_poll(load_poll);
+    Row<7>::fill_load_poll(load_poll);
+    Row<8>::fill_load_poll(load_poll);
   }
 };
+const Table& table() {
+  static const Table t;
+  return t;
+}
 }  // namespace
 
 const void* kernel_for(int nranks, int protocol, int op) {
-  static const Table table;
   if (nranks < kMinRanks || nranks > kMaxRanks || protocol < kLL || protocol >= kNumProtocols || op < 0 || op > 1)
     return nullptr;
-  return table.t[nranks][protocol][op];
+  return table().t[nranks][protocol][op];
+}
+
+const void* launch_kernel_for(int nranks, int protocol, int op, uint64_t count) {
+  if (protocol == kSentinel && sentinel_load_poll(nranks, count) && nranks >= kMinRanks && nranks <= kMaxRanks &&
+      op >= 0 && op <= 1)
+    return table().load_poll[nranks][op];
+  return kernel_for(nranks, protocol, op);
 }
 
 uint64_t slot_bytes_gpu(int protocol, uint64_t count, int n) {

@@ -7,6 +7,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <new>
 #include <vector>
 
 #include "sfc.h"
@@ -43,7 +44,8 @@ struct sfc_ctx {
   uint64_t launches = 0;
   sfc_cost_model model{};
 
-  int occupancy[kNumProtocols][2][2] = {};  // blocks per SM, per (protocol, op, CTA size), 0 = unknown
+  int occupancy[kNumProtocols][2][2][2] = {};  // blocks per SM, per (protocol, op, CTA size, kernel
+                                               // variant), 0 = unknown
   int forced_protocol = 0;                // SFC_PROTOCOL: what AUTO resolves to (0 = the selector)
   int smem_optin = 0;                     // opt-in shared memory per block (bytes)
   int linear_occ[5] = {};                 // fused-linear CTAs per SM: token tile 1/2/4/8, tensor-core (0 = not queried)
@@ -103,10 +105,11 @@ int cta_threads(const sfc_ctx* c, int proto, uint64_t count) {
   return small_msg && (proto == kLL || proto == kSentinel || proto == kLL128Fast) ? kSmallCtaThreads : kThreads;
 }
 
-int occupancy_of(sfc_ctx* c, int proto, int op, int threads) {
-  int& occ = c->occupancy[proto][op][threads == kThreads ? 0 : 1];
+int occupancy_of(sfc_ctx* c, int proto, int op, int threads, uint64_t count) {
+  const void* fn = launch_kernel_for(c->nranks, proto, op, count);
+  const int variant = fn != kernel_for(c->nranks, proto, op) ? 1 : 0;
+  int& occ = c->occupancy[proto][op][threads == kThreads ? 0 : 1][variant];
   if (occ == 0) {
-    const void* fn = kernel_for(c->nranks, proto, op);
     int nb = 0;
     if (fn == nullptr || !cuda_ok(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, threads, 0)))
       return 0;
@@ -120,7 +123,7 @@ int occupancy_of(sfc_ctx* c, int proto, int op, int threads) {
 // all N * G CTAs are co-resident.
 int choose_G(sfc_ctx* c, int proto, int op, uint64_t count, int* gmax_out) {
   const int threads = cta_threads(c, proto, count);
-  const int occ = occupancy_of(c, proto, op, threads);
+  const int occ = occupancy_of(c, proto, op, threads, count);
   const int gmax = std::min(kBarStride, occ * c->sm_count / c->nranks);
   if (gmax_out) *gmax_out = gmax;
   if (gmax <= 0) return 0;
@@ -179,7 +182,7 @@ void fill_common(sfc_ctx* c, KParams& p, int proto, uint64_t count, int k_ops, u
 }
 
 sfc_status launch(sfc_ctx* c, int proto, int op, KParams& p, cudaStream_t stream) {
-  const void* fn = kernel_for(c->nranks, proto, op);
+  const void* fn = launch_kernel_for(c->nranks, proto, op, p.count);
   if (fn == nullptr) return SFC_ERR_UNSUPPORTED;
   int gmax = 0;
   (void)choose_G(c, proto, op, p.count, &gmax);
@@ -208,15 +211,8 @@ sfc_status prepare_timings(uint64_t* timings, int k_ops, cudaStream_t stream) {
 // (In device-epoch mode 0 stays 0: the kernel reads the epoch.)
 uint32_t resolve_epoch(const sfc_ctx* c, uint32_t e) { return e == 0 && !c->cfg.device_epochs ? c->next_epoch : e; }
 
-sfc_status one_op(sfc_ctx* c, sfc_op op, const void* const* in, void* const* out, size_t count, sfc_dtype dtype,
-                  sfc_protocol protocol, uint32_t epoch, void* stream) {
-  if (c == nullptr || in == nullptr || out == nullptr) return SFC_ERR_INVALID;
-  epoch = resolve_epoch(c, epoch);
-  if (count == 0) return (dtype == SFC_BF16) ? SFC_OK : SFC_ERR_UNSUPPORTED;
-  int proto = protocol;
-  if (proto == SFC_PROTO_AUTO) proto = sfc_select_protocol(c, op, count * 2, c->nranks);
-  sfc_status s = check_common(c, op, count, dtype, proto, epoch, 1);
-  if (s != SFC_OK) return s;
+// Operand checks of a single operation (pointers, alignment, no overlap).
+sfc_status check_operands(const sfc_ctx* c, sfc_op op, const void* const* in, void* const* out, size_t count) {
   const int N = c->nranks;
   const size_t in_bytes = count * 2;
   const size_t out_bytes = (op == SFC_OP_ALLGATHER ? N : 1) * count * 2;
@@ -229,6 +225,21 @@ sfc_status one_op(sfc_ctx* c, sfc_op op, const void* const* in, void* const* out
       if (a < b && overlap(out[a], out_bytes, out[b], out_bytes)) return SFC_ERR_INVALID;
     }
   }
+  return SFC_OK;
+}
+
+sfc_status one_op(sfc_ctx* c, sfc_op op, const void* const* in, void* const* out, size_t count, sfc_dtype dtype,
+                  sfc_protocol protocol, uint32_t epoch, void* stream) {
+  if (c == nullptr || in == nullptr || out == nullptr) return SFC_ERR_INVALID;
+  epoch = resolve_epoch(c, epoch);
+  if (count == 0) return (dtype == SFC_BF16) ? SFC_OK : SFC_ERR_UNSUPPORTED;
+  int proto = protocol;
+  if (proto == SFC_PROTO_AUTO) proto = sfc_select_protocol(c, op, count * 2, c->nranks);
+  sfc_status s = check_common(c, op, count, dtype, proto, epoch, 1);
+  if (s != SFC_OK) return s;
+  s = check_operands(c, op, in, out, count);
+  if (s != SFC_OK) return s;
+  const int N = c->nranks;
   KParams p{};
   for (int r = 0; r < N; ++r) {
     p.in_inline[r] = static_cast<const uint16_t*>(in[r]);
@@ -573,6 +584,78 @@ sfc_status sfc_allreduce(sfc_ctx* c, const void* const* in, void* const* out, si
 sfc_status sfc_allgather(sfc_ctx* c, const void* const* in, void* const* out, size_t count, sfc_dtype dtype,
                          sfc_protocol protocol, uint32_t epoch, void* stream) {
   return one_op(c, SFC_OP_ALLGATHER, in, out, count, dtype, protocol, epoch, stream);
+}
+
+// A prepared single operation: checks, protocol, kernel and launch shape
+// fixed once; a launch only takes the next epoch and launches.
+struct sfc_plan {
+  sfc_ctx* c = nullptr;
+  const void* fn = nullptr;
+  int grid = 0;
+  int block = 0;
+  KParams p{};
+};
+
+sfc_status sfc_plan_create(sfc_ctx* c, sfc_op op, const void* const* in, void* const* out, size_t count,
+                           sfc_dtype dtype, sfc_protocol protocol, sfc_plan** plan) {
+  if (plan == nullptr) return SFC_ERR_INVALID;
+  *plan = nullptr;
+  if (c == nullptr || in == nullptr || out == nullptr || count == 0) return SFC_ERR_INVALID;
+  int proto = protocol;
+  if (proto == SFC_PROTO_AUTO) proto = sfc_select_protocol(c, op, count * 2, c->nranks);
+  sfc_status s = check_common(c, op, count, dtype, proto, c->cfg.device_epochs ? 0 : c->next_epoch, 1);
+  if (s != SFC_OK) return s;
+  s = check_operands(c, op, in, out, count);
+  if (s != SFC_OK) return s;
+  const void* fn = launch_kernel_for(c->nranks, proto, op, count);
+  if (fn == nullptr) return SFC_ERR_UNSUPPORTED;
+  int gmax = 0;
+  const int G = choose_G(c, proto, op, count, &gmax);
+  if (G < 1 || G > gmax) return SFC_ERR_RESOURCES;
+  sfc_plan* pl = new (std::nothrow) sfc_plan();
+  if (pl == nullptr) return SFC_ERR_RESOURCES;
+  pl->c = c;
+  pl->fn = fn;
+  pl->grid = c->nranks * G;
+  pl->block = cta_threads(c, proto, count);
+  for (int r = 0; r < c->nranks; ++r) {
+    pl->p.in_inline[r] = static_cast<const uint16_t*>(in[r]);
+    pl->p.out_inline[r] = static_cast<uint16_t*>(out[r]);
+  }
+  pl->p.addr_mode = 0;
+  fill_common(c, pl->p, proto, count, 1, 0, G);
+  *plan = pl;
+  return SFC_OK;
+}
+
+sfc_status sfc_plan_launch(sfc_plan* pl, void* stream) {
+  if (pl == nullptr) return SFC_ERR_INVALID;
+  sfc_ctx* c = pl->c;
+  if (c->poisoned) return SFC_ERR_ABORTED;
+  uint32_t e = 0;
+  if (!c->cfg.device_epochs) {
+    e = c->next_epoch;
+    if (e == 0) return SFC_ERR_EPOCH;  // the sequence is spent: sfc_reset first
+  }
+  pl->p.first_epoch = e;
+  pl->p.silent_rank = c->silent_rank;
+  void* args[] = {&pl->p};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const cudaError_t err = cudaLaunchCooperativeKernel(pl->fn, dim3(pl->grid), dim3(pl->block), args, 0, st);
+  if (err == cudaErrorCooperativeLaunchTooLarge) {
+    (void)cudaGetLastError();
+    return SFC_ERR_RESOURCES;
+  }
+  if (!cuda_ok(err)) return SFC_ERR_CUDA;
+  c->launches++;
+  c->last_stream = st;
+  if (!c->cfg.device_epochs) c->next_epoch = e + 1;
+  return SFC_OK;
+}
+
+sfc_status sfc_plan_destroy(sfc_plan* pl) {
+  delete pl;
+  return SFC_OK;
 }
 
 sfc_status sfc_allreduce_chain(sfc_ctx* c, int k_ops, const void* const* in_table, void* const* out_table,

@@ -40,9 +40,13 @@ def _percentile(v, q):
     return float(v[min(len(v) - 1, max(0, int(round(q * (len(v) - 1)))))]) if v else float("nan")
 
 
-def measure_point(comm, op, proto, count, k_ops, reps, gen, dev):
+def measure_point(comm, op, proto, count, k_ops, reps, gen, dev, distinct=None):
+    """p50 / p99 per operation of `reps` chains of k_ops operations (after one
+    warm-up chain). Operations cycle through `distinct` inputs per rank
+    (default min(k_ops, 8)); more distinct inputs than fit in L2 make every
+    chain read its inputs from HBM."""
     n = comm.nranks
-    distinct = min(k_ops, 8)
+    distinct = min(k_ops, 8) if distinct is None else max(1, min(k_ops, int(distinct)))
     stride = (count + 7) // 8 * 8
     xin = torch.randn(distinct * n * stride, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
     out_count = count if op == "allreduce" else n * count

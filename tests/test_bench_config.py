@@ -58,3 +58,35 @@ def test_recorded_traffic_is_keyed_on_device_sources_and_launch_shape(monkeypatc
     assert b.recorded_traffic(key, grid=ent["grid"], block=ent["block"]) is None
     for rel in b.KERNEL_SOURCES:
         assert os.path.exists(os.path.join(ROOT, rel)), rel
+
+
+def test_large_target_points_read_their_inputs_from_hbm():
+    b = _bench()
+    for n in b.TARGET_RANKS:
+        for nbytes in b.TARGET_LARGE:
+            k = b.large_point_inputs(n, nbytes)
+            assert 8 <= k <= 128
+            total = k * n * nbytes
+            assert total <= (3 << 29) or k == 8          # bounded device memory
+            assert total >= 2 * b.L2_BYTES or k == 128   # inputs twice the L2 unless capped
+
+
+def test_ncu_record_parses_a_launch_list(tmp_path, monkeypatch):
+    from latency_self_synchronizing_b200 import ncu_record
+
+    hdr = '"ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream","Block Size",' \
+          '"Grid Size","Device","CC","Section Name","Metric Name","Metric Unit","Metric Value"\n'
+    rows = []
+    for lid, (name, grid) in enumerate([("void sfc::sfc_kernel<4, 3, 0>(sfc::KParams)", 32),
+                                        ("void other_kernel(int)", 1)]):
+        for metric, unit, val in [("dram__bytes_read.sum", "Mbyte", "10.5"), ("dram__bytes_write.sum", "Kbyte", "500"),
+                                  ("gpu__time_duration.sum", "usecond", "278.5")]:
+            rows.append(f'"{lid}","1","python","h","{name}","1","7","(128, 1, 1)","({grid}, 1, 1)","0","10.0",'
+                        f'"Command line profiler metrics","{metric}","{unit}","{val}"\n')
+    p = tmp_path / "launches.csv"
+    p.write_text("==PROF== noise\n" + hdr + "".join(rows))
+    got = ncu_record.read_launches(str(p))
+    assert len(got) == 1  # only the chain kernels
+    assert got[0]["grid"] == 32 and got[0]["block"] == 128
+    assert got[0]["dram_bytes"] == 10.5e6 + 500e3
+    assert got[0]["duration_us"] == 278.5

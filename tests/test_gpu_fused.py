@@ -1,13 +1,9 @@
-"""The fused row-parallel linear + all-reduce (one decode token) against an
-fp64 reference of the same product and sum.
-
-The partial products are fp32 accumulations whose order is the kernel's, so
-they are not bit-exact to any plain definition; the all-reduce of them is.
-Bound used (per output element): each rank's partial p_r is within
-2^-8 |d_r| + kdim 2^-24 a_r of the exact dot product d_r (one bf16 rounding,
-kdim fp32 roundings of partial sums bounded by a_r = sum_i |W_ri x_ri|), and
-the rank-order all-reduce of the partials is within 2^-7 N sum_r |p_r| of
-their exact sum. Every rank's output must be bit-identical.
+"""The fused row-parallel linear + all-reduce against the oracle
+(oracle/linear.py): the exact value of the layer and the error bound of any
+implementation that accumulates each partial in fp32 in its own order, rounds
+it to bf16 and all-reduces the partials by the rank-order fold. The partial
+products are fp32 accumulations whose order is the kernel's, so they are not
+bit-exact to any plain definition; every rank's output must be bit-identical.
 """
 import numpy as np
 import pytest
@@ -15,6 +11,7 @@ import torch
 
 from latency_self_synchronizing_b200 import api
 from latency_self_synchronizing_b200.inputs import make_inputs
+from oracle import linear
 from oracle.bf16 import bf16_bits_to_f32
 
 pytestmark = pytest.mark.gpu
@@ -48,14 +45,10 @@ def test_linear_allreduce_within_bound(n, hidden, kdim):
             ys = [Y[r].cpu().view(torch.int16).numpy().view(np.uint16) for r in range(n)]
             for r in range(1, n):
                 np.testing.assert_array_equal(ys[r], ys[0])
-            wf = bf16_bits_to_f32(w).astype(np.float64)
-            xf = bf16_bits_to_f32(x).astype(np.float64)
-            d = np.einsum("rhk,rk->rh", wf, xf)               # exact enough in fp64
-            a = np.einsum("rhk,rk->rh", np.abs(wf), np.abs(xf))
-            eps = 2.0 ** -8 * np.abs(d) + kdim * 2.0 ** -24 * a
-            bound = eps.sum(0) + 2.0 ** -7 * n * (np.abs(d) + eps).sum(0)
+            exact = linear.linear_allreduce_fp64(w, x)[0]
+            bound = linear.linear_allreduce_error_bound(w, x)[0]
             got = bf16_bits_to_f32(ys[0]).astype(np.float64)
-            assert np.all(np.abs(got - d.sum(0)) <= bound)
+            assert np.all(np.abs(got - exact) <= bound)
     finally:
         comm.close()
 
@@ -108,13 +101,9 @@ def test_linear_allreduce_tokens_within_bound(n, hidden, kdim, tokens):
             ys = [Y[r].cpu().view(torch.int16).numpy().view(np.uint16) for r in range(n)]
             for r in range(1, n):
                 np.testing.assert_array_equal(ys[r], ys[0])
-            wf = bf16_bits_to_f32(w).astype(np.float64)
-            xf = bf16_bits_to_f32(x).astype(np.float64)
-            d = np.einsum("rhk,rtk->rth", wf, xf)
-            a = np.einsum("rhk,rtk->rth", np.abs(wf), np.abs(xf))
-            eps = 2.0 ** -8 * np.abs(d) + kdim * 2.0 ** -24 * a
-            bound = eps.sum(0) + 2.0 ** -7 * n * (np.abs(d) + eps).sum(0)
-            got = bf16_bits_to_f32(ys[0]).astype(np.float64)
-            assert np.all(np.abs(got - d.sum(0)) <= bound)
+            exact = linear.linear_allreduce_fp64(w, x)
+            bound = linear.linear_allreduce_error_bound(w, x)
+            got = bf16_bits_to_f32(ys[0]).reshape(tokens, hidden).astype(np.float64)
+            assert np.all(np.abs(got - exact) <= bound)
     finally:
         comm.close()

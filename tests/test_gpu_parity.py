@@ -244,31 +244,72 @@ def test_workload_decode_h4096_full(proto, tokens):
 
 @pytest.mark.parametrize("proto", AR_PROTOS)
 @pytest.mark.parametrize("n", [2, 8])
-def test_sweep_large_sizes_sampled(proto, n):
-    """Up to 64 MB per rank: every output compared at sampled indices."""
-    for nbytes in (1 << 20, 64 << 20):
-        count = nbytes // 2
+def test_sweep_1mb_every_element(proto, n):
+    """1 MB per rank (where the selector hands over to the barrier kernels):
+    every element of every rank compared with the closed form."""
+    count = (1 << 20) // 2
+    comm = api.Communicator(n, 1 << 20, protocols=[proto])
+    try:
+        x = make_inputs(seed=(1 << 20) + n, k_ops=2, nranks=n, count=count)
+        _assert_ar(run_chain(comm, proto, x), x)
+    finally:
+        comm.close()
+        torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("n", [2, 4, 8])
+def test_selected_protocol_16mb_every_element(n):
+    """16 MB per rank with the protocol the selector picks there (and at
+    1 MB): every element compared with the closed form."""
+    nbytes = 16 << 20
+    count = nbytes // 2
+    probe = api.Communicator(n, 1 << 10)  # every protocol provisioned: the selector's own choice
+    try:
+        chosen = {probe.select_protocol("allreduce", b, n).name.lower() for b in (1 << 20, nbytes)}
+    finally:
+        probe.close()
+    x = make_inputs(seed=nbytes + n, k_ops=2, nranks=n, count=count)
+    want = _want_ar(x)
+    for proto in sorted(chosen):
         comm = api.Communicator(n, nbytes, protocols=[proto])
         try:
-            x = make_inputs(seed=nbytes + n, k_ops=2, nranks=n, count=count)
             out = run_chain(comm, proto, x)
-            idx = np.unique(np.concatenate([np.arange(64), count - 64 + np.arange(64),
-                                            np.random.default_rng(n).integers(0, count, 4096)]))
-            for k in range(2):
-                want = reference.allreduce(x[k][:, idx])
-                for r in range(n):
-                    np.testing.assert_array_equal(out[k, r, idx], want)
+            for r in range(n):
+                np.testing.assert_array_equal(out[:, r, :], want, err_msg=f"{proto} rank {r}")
         finally:
             comm.close()
             torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("proto", AR_PROTOS)
+@pytest.mark.parametrize("n", [2, 8])
+def test_sweep_64mb_sampled(proto, n):
+    """64 MB per rank: every output compared at sampled indices (the head,
+    the tail and 4096 random positions)."""
+    nbytes = 64 << 20
+    count = nbytes // 2
+    comm = api.Communicator(n, nbytes, protocols=[proto])
+    try:
+        x = make_inputs(seed=nbytes + n, k_ops=2, nranks=n, count=count)
+        out = run_chain(comm, proto, x)
+        idx = np.unique(np.concatenate([np.arange(64), count - 64 + np.arange(64),
+                                        np.random.default_rng(n).integers(0, count, 4096)]))
+        for k in range(2):
+            want = reference.allreduce(x[k][:, idx])
+            for r in range(n):
+                np.testing.assert_array_equal(out[k, r, idx], want)
+    finally:
+        comm.close()
+        torch.cuda.empty_cache()
+
+
 @pytest.mark.parametrize("proto", AG_PROTOS)
 def test_workload_allgather_with_skew(proto):
-    """8 ranks, shards 512 B .. 1 MB subset, uniform[-4,4), exponential start
-    skew (mean 2 us) per (op, rank); outputs bit-identical across 5 skew seeds."""
+    """8 ranks, every shard size 512 B .. 1 MB (powers of two), uniform[-4,4),
+    exponential start skew (mean 2 us) per (op, rank); outputs equal to the
+    closed form and bit-identical across 5 skew seeds."""
     n = 8
-    for nbytes in (512, 16384, 1 << 20):
+    for nbytes in [512 << i for i in range(12)]:
         count = nbytes // 2
         comm = api.Communicator(n, nbytes)
         try:
