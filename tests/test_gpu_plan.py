@@ -62,8 +62,9 @@ def test_plan_allgather_and_argument_checks():
         assert comm.status()[0] == api.Status.OK
         for r in range(n):
             np.testing.assert_array_equal(_bits(outs[r]), reference.allgather(x))
+        ar_outs = [torch.empty(count, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
         with pytest.raises(api.SfcError) as ei:  # an output that overlaps an input
-            comm.plan(ins, [ins[0]] + outs[1:], op="allreduce", protocol="ll")
+            comm.plan(ins, [ins[0]] + ar_outs[1:], op="allreduce", protocol="ll")
         assert ei.value.status == api.Status.INVALID
         with pytest.raises(api.SfcError) as ei:  # allgather has no twoshot
             comm.plan(ins, outs, op="allgather", protocol="barrier_twoshot")
