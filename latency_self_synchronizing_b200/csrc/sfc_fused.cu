@@ -46,6 +46,21 @@ SFC_DEV uint4 ld_stream_v4(const void* p) {
   return v;
 }
 
+// x_r into shared memory: every thread issues its 16-byte asynchronous
+// copies (global -> shared, no register round trip) before waiting for any,
+// so the whole activation is in flight at once instead of one load per
+// thread and loop trip. `bytes` is a multiple of 16; both addresses 16-byte
+// aligned. The caller synchronizes the block afterwards.
+SFC_DEV void copy_to_smem_async(void* dst, const void* src, uint64_t bytes) {
+  const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  const char* s = static_cast<const char*>(src);
+#pragma unroll 1
+  for (uint64_t o = static_cast<uint64_t>(threadIdx.x) * 16; o < bytes; o += static_cast<uint64_t>(blockDim.x) * 16)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(base + static_cast<uint32_t>(o)), "l"(s + o)
+                 : "memory");
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // acc + w0 x0 + w1 x1 + ... + w7 x7, one fp32 FMA per element in element
 // order, each taking its two bf16 operands as they are (sm_100's mixed
 // bf16 x bf16 + f32 FMA: the same exact-product, single-rounding step as
@@ -249,10 +264,7 @@ __global__ void __launch_bounds__(kLinearThreads, 2) linear_mma_kernel(const __g
   uint4* ownv = reinterpret_cast<uint4*>(parts + static_cast<uint64_t>(per) * ks * 128);
   uint32_t* cnt = reinterpret_cast<uint32_t*>(ownv + static_cast<uint64_t>(per) * 16);
 
-  for (uint64_t i = threadIdx.x; i < tokens * kdim / 8; i += blockDim.x) {
-    const uint64_t u = i / (kdim / 8), c = i - u * (kdim / 8);
-    reinterpret_cast<uint4*>(xs)[i] = ld_nc_v4(p.x[r] + u * kdim + c * 8);
-  }
+  copy_to_smem_async(xs, p.x[r], static_cast<uint64_t>(tokens) * kdim * 2);
   for (uint32_t i = threadIdx.x; i < per; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
 
