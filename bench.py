@@ -267,7 +267,9 @@ def measure_targets(dev, floor_us, peak_gbs, large_only=False):
             k = large_point_inputs(n, b)
             comm = api.Communicator(n, b, protocols=[proto])
             try:
+                torch.cuda.nvtx.range_push("targets_large")  # the launches an ncu traffic capture records
                 pt = sweep.measure_point(comm, "allreduce", proto, b // 2, k, 3, gen, dev, distinct=k)
+                torch.cuda.nvtx.range_pop()
                 shape = comm.launch_shape("allreduce", proto, b // 2)
             finally:
                 comm.close()
@@ -368,9 +370,11 @@ def run_gpu(args):
     wall0 = torch.cuda.Event(enable_timing=True)
     wall1 = torch.cuda.Event(enable_timing=True)
     wall0.record(stream)
+    torch.cuda.nvtx.range_push("timed")  # ncu captures select this range (--nvtx --nvtx-include timed/)
     for s in range(args.steps):
         l2_flush.zero_()
         step(tims[s], evs[s])
+    torch.cuda.nvtx.range_pop()
     wall1.record(stream)
     torch.cuda.synchronize()
     if ws > 1:

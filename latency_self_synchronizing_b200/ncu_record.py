@@ -8,11 +8,12 @@ metrics dram__bytes_read.sum, dram__bytes_write.sum and gpu__time_duration.sum
 of the chain kernels (`-k regex:sfc_kernel`):
 
 * bench: `python bench.py --steps 2 --warmup 3 --no-cpu-baseline --no-targets`
-  captured with `-s 12 -c 4` (the first timed step: one chain launch per
-  token count);
-* targets: `python bench.py --targets-only --large-only`, every launch (per
-  large point one warm-up chain and three timed chains, points in the order
-  the bench measures them).
+  captured with `--nvtx --nvtx-include timed/ -c 4` (the first timed step:
+  one chain launch per token count);
+* targets: `python bench.py --targets-only --large-only` captured with
+  `--nvtx --nvtx-include targets_large/`, every launch (per large point one
+  warm-up chain and three timed chains, points in the order the bench
+  measures them).
 
 The entries are keyed as bench.py looks them up (kernel, operations, bytes
 per rank, grid, block) and stamped with the current kernel-source hash, so
@@ -99,8 +100,8 @@ def record_bench(path):
         entries[key] = {"dram_bytes_per_launch": la["dram_bytes"], "duration_us_under_ncu": la["duration_us"],
                         "grid": la["grid"], "block": la["block"]}
     _save(entries, "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum "
-                   "--clock-control none -k regex:sfc_kernel -s 12 -c 4 --csv --log-file LAUNCHES.csv "
-                   "python bench.py --steps 2 --warmup 3 --no-cpu-baseline --no-targets")
+                   "--clock-control none --nvtx --nvtx-include timed/ -k regex:sfc_kernel -c 4 --csv "
+                   "--log-file LAUNCHES.csv python bench.py --steps 2 --warmup 3 --no-cpu-baseline --no-targets")
     return entries
 
 
@@ -124,8 +125,8 @@ def record_targets(path):
                         "duration_us_under_ncu": statistics.median(x["duration_us"] for x in group),
                         "grid": group[0]["grid"], "block": group[0]["block"]}
     _save(entries, "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum "
-                   "--clock-control none -k regex:sfc_kernel --csv --log-file LAUNCHES.csv "
-                   "python bench.py --targets-only --large-only")
+                   "--clock-control none --nvtx --nvtx-include targets_large/ -k regex:sfc_kernel --csv "
+                   "--log-file LAUNCHES.csv python bench.py --targets-only --large-only")
     return entries
 
 
