@@ -74,3 +74,11 @@ def test_odd_rank_counts_under_skew(proto, n):
     """Rank counts the power-of-two cases do not reach (uneven twoshot shards,
     source indices that skip the own rank at every position), ragged size."""
     _run(proto, n=n, count=777, total_ops=1 << 15, skew_mean_ns=500.0, seed=20 + n)
+
+
+@pytest.mark.parametrize("n,count", [(8, 32769), (4, 80000), (2, 262147)])
+def test_sentinel_load_polls_under_skew(n, count):
+    """Large sentinel messages ((N - 1) x bytes >= 448 KB) poll with loads and
+    reset with stores behind a release fence: the resets must land before a
+    writer reuses the slot two epochs later, under changing arrival orders."""
+    _run("sentinel", n=n, count=count, total_ops=1 << 13, skew_mean_ns=2000.0, seed=30 + n)
