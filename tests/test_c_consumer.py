@@ -52,6 +52,12 @@ def _program():
     lines.append("  sfc_ctx* ctx = NULL;")
     lines.append('  printf("init_bad_ranks %d\\n", (int)sfc_init(&ctx, 1, 4096, NULL));')
     lines.append('  printf("destroy_null %d\\n", (int)sfc_destroy(NULL));')
+    lines.append("  sfc_plan* plan = (sfc_plan*)1;")
+    lines.append('  printf("plan_create_null %d\\n", (int)sfc_plan_create(NULL, SFC_OP_ALLREDUCE, NULL, NULL, 8, SFC_BF16,'
+                 ' SFC_PROTO_LL, &plan));')
+    lines.append('  printf("plan_cleared %d\\n", plan == NULL);')
+    lines.append('  printf("plan_launch_null %d\\n", (int)sfc_plan_launch(NULL, NULL));')
+    lines.append('  printf("plan_destroy_null %d\\n", (int)sfc_plan_destroy(NULL));')
     lines += ["  return 0;", "}"]
     return "\n".join(lines) + "\n"
 
@@ -106,6 +112,9 @@ def test_selector_and_bytes_agree_with_the_binding(c_output):
 
 
 def test_argument_checks_from_c(c_output):
-    vals = {k: int(v) for k, v in c_output if k in ("init_null", "init_bad_ranks", "destroy_null")}
+    keys = ("init_null", "init_bad_ranks", "destroy_null", "plan_create_null", "plan_cleared", "plan_launch_null",
+            "plan_destroy_null")
+    vals = {k: int(v) for k, v in c_output if k in keys}
     assert vals == {"init_null": int(api.Status.INVALID), "init_bad_ranks": int(api.Status.INVALID),
-                    "destroy_null": int(api.Status.INVALID)}
+                    "destroy_null": int(api.Status.INVALID), "plan_create_null": int(api.Status.INVALID),
+                    "plan_cleared": 1, "plan_launch_null": int(api.Status.INVALID), "plan_destroy_null": 0}
