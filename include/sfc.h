@@ -53,9 +53,12 @@
  *     NULL = the legacy default stream). Calls on one context must be
  *     ordered on the GPU (one stream, or streams joined by events).
  *   - Device-side errors (a wait that ran out, a sentinel in an input under
- *     debug checks) are sticky: the kernel records them and every later
- *     kernel of the context exits at once, until sfc_reset. They are read
- *     with sfc_get_status.
+ *     debug checks) are sticky: the kernel records them, every later
+ *     chain launch of the context exits at once and every later single
+ *     operation at its first wait check (a single operation does not load
+ *     the error word before its first push, which would cost it an L2 round
+ *     trip), until sfc_reset; the host refuses new work once sfc_get_status
+ *     has seen the error. They are read with sfc_get_status.
  */
 #ifndef SFC_H
 #define SFC_H

@@ -141,6 +141,7 @@ class Communicator:
         self._device = torch.cuda.current_device()
         self._ptrs_in = (C.c_void_p * self.nranks)()
         self._ptrs_out = (C.c_void_p * self.nranks)()
+        self._last = None  # (op, inputs, outputs, data pointers) of the last single call that passed the checks
         self._plans = []
 
     # ----------------------------------------------------------- lifecycle
@@ -190,29 +191,44 @@ class Communicator:
         # per-call cost matters here (one launch per all-reduce): checks are
         # plain attribute reads, the pointer arrays are reused, the epoch is
         # left to the library (0 = next) and the stream read without a
-        # Stream object
+        # Stream object. A call on the same tensor objects as the last one,
+        # still at the same addresses and sizes (a decode loop on fixed
+        # buffers), skips the metadata checks: they passed for these tensors.
         n = self.nranks
-        if len(inputs) != n or len(outputs) != n:
-            raise ValueError(f"need {n} inputs and {n} outputs")
+        last = self._last
+        ptrs = None
+        if last is not None and last[0] == op and len(inputs) == n and len(outputs) == n:
+            li, lo, lp = last[1], last[2], last[3]
+            if all(a is b for a, b in zip(inputs, li)) and all(a is b for a, b in zip(outputs, lo)):
+                ptrs = [(t.data_ptr(), t.numel()) for t in inputs] + [(t.data_ptr(), t.numel()) for t in outputs]
+                if ptrs != lp:
+                    ptrs = None
         count = inputs[0].numel()
-        want_out = count if op == Op.ALLREDUCE else n * count
+        if ptrs is None:
+            self._last = None
+            if len(inputs) != n or len(outputs) != n:
+                raise ValueError(f"need {n} inputs and {n} outputs")
+            want_out = count if op == Op.ALLREDUCE else n * count
+            ins, outs = self._ptrs_in, self._ptrs_out
+            bf16 = torch.bfloat16
+            dev = self._device
+            for r in range(n):
+                a, b = inputs[r], outputs[r]
+                if not (a.is_cuda and b.is_cuda and a.dtype is bf16 and b.dtype is bf16 and a.is_contiguous()
+                        and b.is_contiguous()):
+                    _dev_ptr(a, "input")
+                    _dev_ptr(b, "output")
+                if a.get_device() != dev or b.get_device() != dev:
+                    raise ValueError(f"operands must be on cuda:{dev}, the communicator's device")
+                if a.numel() != count:
+                    raise ValueError("all inputs must have the same number of elements")
+                if b.numel() != want_out:
+                    raise ValueError(f"outputs must have {want_out} elements")
+                ins[r] = a.data_ptr()
+                outs[r] = b.data_ptr()
+            self._last = (op, tuple(inputs), tuple(outputs),
+                          [(t.data_ptr(), t.numel()) for t in inputs] + [(t.data_ptr(), t.numel()) for t in outputs])
         ins, outs = self._ptrs_in, self._ptrs_out
-        bf16 = torch.bfloat16
-        dev = self._device
-        for r in range(n):
-            a, b = inputs[r], outputs[r]
-            if not (a.is_cuda and b.is_cuda and a.dtype is bf16 and b.dtype is bf16 and a.is_contiguous()
-                    and b.is_contiguous()):
-                _dev_ptr(a, "input")
-                _dev_ptr(b, "output")
-            if a.get_device() != dev or b.get_device() != dev:
-                raise ValueError(f"operands must be on cuda:{dev}, the communicator's device")
-            if a.numel() != count:
-                raise ValueError("all inputs must have the same number of elements")
-            if b.numel() != want_out:
-                raise ValueError(f"outputs must have {want_out} elements")
-            ins[r] = a.data_ptr()
-            outs[r] = b.data_ptr()
         proto = protocol if type(protocol) is int else int(as_protocol(protocol))
         e = 0 if epoch is None else int(epoch)
         rc = fn(self._ctx, ins, outs, count, 0, proto, e, _stream_handle(stream, self._device))

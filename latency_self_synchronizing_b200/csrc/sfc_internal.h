@@ -111,6 +111,7 @@ struct KParams {
   uint64_t timeout_ns;
   int debug;
   int silent_rank;      // -1 = none
+  int skip_abort_prologue;  // nonzero (single operations of a context): no abort-word load before the first push
 };
 
 // Fused row-parallel linear + LL all-reduce (one decode token).

@@ -248,6 +248,7 @@ sfc_status one_op(sfc_ctx* c, sfc_op op, const void* const* in, void* const* out
   p.addr_mode = 0;
   const int G = choose_G(c, proto, op, count, nullptr);
   fill_common(c, p, proto, count, 1, epoch, G);
+  p.skip_abort_prologue = 1;
   s = launch(c, proto, op, p, static_cast<cudaStream_t>(stream));
   if (s == SFC_OK && !c->cfg.device_epochs) c->next_epoch = epoch + 1;
   return s;
@@ -624,6 +625,7 @@ sfc_status sfc_plan_create(sfc_ctx* c, sfc_op op, const void* const* in, void* c
   }
   pl->p.addr_mode = 0;
   fill_common(c, pl->p, proto, count, 1, 0, G);
+  pl->p.skip_abort_prologue = 1;
   *plan = pl;
   return SFC_OK;
 }

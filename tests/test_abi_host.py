@@ -199,6 +199,7 @@ def _bare_communicator(n=2):
     c = api.Communicator.__new__(api.Communicator)
     c.nranks, c._device, c._ctx, c._lib = n, 0, None, NoCalls()
     c._ptrs_in, c._ptrs_out = [None] * n, [None] * n
+    c._last, c._plans = None, []
     return c
 
 

@@ -71,3 +71,35 @@ def test_plan_allgather_and_argument_checks():
         assert ei.value.status == api.Status.UNSUPPORTED
     finally:
         comm.close()
+
+
+def test_repeated_single_calls_on_the_same_tensors():
+    """The binding skips its metadata checks when a call repeats the last
+    call's tensor objects at the same addresses and sizes; any change makes
+    it check again."""
+    n, count = 4, 2048
+    comm = api.Communicator(n, 2 * 4 * count)
+    try:
+        x = make_inputs(seed=77, k_ops=2, nranks=n, count=count)
+        ins = [_dev(x[0, r]) for r in range(n)]
+        outs = [torch.empty(count, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+        for k in range(2):
+            for r in range(n):
+                ins[r].copy_(_dev(x[k, r]))
+            comm.allreduce(ins, outs, protocol="ll")  # the second call takes the short path
+            torch.cuda.synchronize()
+            for r in range(n):
+                np.testing.assert_array_equal(_bits(outs[r]), reference.allreduce(x[k]))
+        with pytest.raises(TypeError, match="CUDA"):  # another object: checked again
+            comm.allreduce(ins, outs[:-1] + [torch.empty(count, dtype=torch.bfloat16)], protocol="ll")
+        comm.allreduce(ins, outs, protocol="ll")
+        outs[0].resize_(count // 2)  # same object, new size: checked again
+        with pytest.raises(ValueError):
+            comm.allreduce(ins, outs, protocol="ll")
+        ins[1].resize_(count // 2)
+        with pytest.raises(ValueError):
+            comm.allreduce(ins, outs, protocol="ll")
+        torch.cuda.synchronize()
+        assert comm.status()[0] == api.Status.OK
+    finally:
+        comm.close()
