@@ -54,7 +54,7 @@ def test_million_ops_under_skew(proto):
     _run(proto, n=4, count=1000, total_ops=1_000_000, skew_mean_ns=300.0, seed=7)
 
 
-@pytest.mark.parametrize("proto", ["ll", "sentinel", "barrier_oneshot", "barrier_oneshot_db", "barrier_twoshot"])
+@pytest.mark.parametrize("proto", ["ll", "sentinel", "ll128", "barrier_oneshot", "barrier_oneshot_db", "barrier_twoshot"])
 def test_many_ops_eight_ranks(proto):
     _run(proto, n=8, count=4099, total_ops=1 << 17, skew_mean_ns=1000.0, seed=8)
 
