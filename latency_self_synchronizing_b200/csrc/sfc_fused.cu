@@ -46,21 +46,6 @@ SFC_DEV uint4 ld_stream_v4(const void* p) {
   return v;
 }
 
-// x_r into shared memory: every thread issues its 16-byte asynchronous
-// copies (global -> shared, no register round trip) before waiting for any,
-// so the whole activation is in flight at once instead of one load per
-// thread and loop trip. `bytes` is a multiple of 16; both addresses 16-byte
-// aligned. The caller synchronizes the block afterwards.
-SFC_DEV void copy_to_smem_async(void* dst, const void* src, uint64_t bytes) {
-  const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
-  const char* s = static_cast<const char*>(src);
-#pragma unroll 1
-  for (uint64_t o = static_cast<uint64_t>(threadIdx.x) * 16; o < bytes; o += static_cast<uint64_t>(blockDim.x) * 16)
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(base + static_cast<uint32_t>(o)), "l"(s + o)
-                 : "memory");
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
-
 // acc + w0 x0 + w1 x1 + ... + w7 x7, one fp32 FMA per element in element
 // order, each taking its two bf16 operands as they are (sm_100's mixed
 // bf16 x bf16 + f32 FMA: the same exact-product, single-rounding step as
@@ -206,19 +191,20 @@ __global__ void __launch_bounds__(kLinearThreads, T >= 8 ? 1 : 2)
 // ---------------------------------------------------------------------------
 // 2..8 tokens on the tensor cores (mma.sync m16n8k16, bf16 in, fp32 out).
 // The tile is 16 rows of W_r (two LL vectors) by 8 token columns (tokens past
-// p.tokens are zero). Columns go in blocks of 32, two MMA steps each, whose
-// k order is a permutation both operands share, chosen so that every thread
-// reads its weights as two 16-byte pieces: thread (group g, quad q) takes
-// W[row0 + g][k0 + 8q .. 8q+7] and W[row0 + g + 8][same]. For the first MMA
-// its A registers are (row g, k0+8q..+1), (row g+8, k0+8q..+1), (row g,
-// k0+8q+2..+3), (row g+8, k0+8q+2..+3), which the instruction reads as the
-// logical columns 2q, 2q+1 / 2q+8, 2q+9; the second MMA takes k0+8q+4..+7 the
-// same way. Its B registers are x[token g] at the same physical columns under
-// the same logical names. A dot product does not depend on the order of its
-// terms' indices, so the MMAs compute W x exactly as a sum over the block's
-// 32 columns (fp32 accumulation). The multiply-adds
-// are far below the tensor pipe's rate; the weight stream still bounds the
-// layer, which is why the legacy warp-level instruction suffices here.
+// p.tokens are zero). The MMA's k order is a permutation both operands share,
+// chosen so that every thread reads its weights as whole 16- or 32-byte
+// pieces: thread (group g, quad q) takes W[row0 + g][k0 + P q .. P q + P-1]
+// and W[row0 + g + 8][same], P = 8 or 16 columns, the block being 4P
+// columns wide. Each 4 consecutive columns c .. c+3 of a thread's piece feed
+// one MMA step: its A registers are (row g, c..c+1), (row g+8, c..c+1),
+// (row g, c+2..c+3), (row g+8, c+2..c+3), which the instruction reads as
+// the logical columns 2q, 2q+1 / 2q+8, 2q+9, and its B registers are
+// x[token g] at the same physical columns under the same logical names. Over
+// the four quads one step covers 16 distinct columns, so the steps compute
+// W x exactly as a sum over the block's columns (fp32 accumulation, in the
+// steps' order). The multiply-adds are far below the tensor pipe's rate; the
+// weight stream bounds the layer, which is why the legacy warp-level
+// instruction suffices here.
 SFC_DEV void mma_16x8x16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                          uint32_t b1) {
   asm volatile(
@@ -228,24 +214,61 @@ SFC_DEV void mma_16x8x16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, u
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-SFC_DEV uint2 ld_stream_v2(const void* p) {
-  uint2 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-  return v;
+// 32 bytes of a weight row (the address 32-byte aligned), streamed once
+SFC_DEV void ld_stream_v8(const void* p, uint32_t (&v)[8]) {
+  asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+               : "l"(p));
 }
 
-// Shared memory: x_r [tokens][kdim] | parts [per][ks][16 rows][8 tokens] fp32 |
-// own [per][2 vectors][8 tokens] (packed bf16) | counters [per]. A CTA owns
-// the 16-row tiles [t0, t0 + per) of its rank; LL vector u * hidden / 8 + v
-// carries rows 8v .. 8v+7 of token u.
-constexpr int kMmaPairs = 8;  // 32-column blocks whose loads are issued before their MMAs (256 B a thread)
-template <int NR>
+// One column block of a thread: its piece of rows g and g + 8 (kWide: 32
+// bytes each, 64-column blocks; else 16 bytes, 32-column blocks).
+template <bool kWide>
+struct MmaBlock {
+  static constexpr int kCols = kWide ? 64 : 32;  // columns per block
+  static constexpr int kRegs = kWide ? 8 : 4;    // registers per row piece
+  static constexpr int kRing = kWide ? 4 : 8;    // blocks in flight per thread: 256 bytes either way
+  SFC_DEV static void load(const uint16_t* src, uint32_t (&v)[kRegs]) {
+    if constexpr (kWide) {
+      ld_stream_v8(src, v);
+    } else {
+      const uint4 t = ld_stream_v4(src);
+      v[0] = t.x, v[1] = t.y, v[2] = t.z, v[3] = t.w;
+    }
+  }
+  // xp: x[token g] at the thread's first column of the block (shared memory)
+  SFC_DEV static void mma(float (&d)[4], const uint32_t (&ra)[kRegs], const uint32_t (&rb)[kRegs],
+                          const uint16_t* xp, bool tok_ok) {
+#pragma unroll
+    for (int h = 0; h < kRegs / 4; ++h) {
+      const uint4 xv = tok_ok ? *reinterpret_cast<const uint4*>(xp + 8 * h) : make_uint4(0, 0, 0, 0);
+      mma_16x8x16(d, ra[4 * h], rb[4 * h], ra[4 * h + 1], rb[4 * h + 1], xv.x, xv.y);
+      mma_16x8x16(d, ra[4 * h + 2], rb[4 * h + 2], ra[4 * h + 3], rb[4 * h + 3], xv.z, xv.w);
+    }
+  }
+};
+
+// Shared memory: x_r [tokens][kdim] | parts [per][ks][16 rows][8 tokens]
+// fp32 | own [per][2 vectors][8 tokens] (packed bf16) | counters [per]. A CTA
+// owns the 16-row tiles [t0, t0 + per) of its rank; LL vector
+// u * hidden / 8 + v carries rows 8v .. 8v+7 of token u. A warp keeps
+// kRing blocks of loads in flight as a rolling ring (block i + kRing is
+// requested as soon as block i's MMAs have read their registers); the first
+// tile's ring is filled before the activation is waited for. (Measured on
+// B200 and dropped: refilling the ring with the next tile's first blocks
+// during a tile's last round, and x rows padded to shift the token rows'
+// banks, each 0.5-2 % slower.) With 32-byte pieces a 32-column rest of the
+// row (kdim % 64 == 32) is one 16-byte-piece block, taken by the tile's last
+// part.
+template <int NR, bool kWide>
 __global__ void __launch_bounds__(kLinearThreads, 2) linear_mma_kernel(const __grid_constant__ LinearParams p) {
+  using B = MmaBlock<kWide>;
+  constexpr int kRing = B::kRing;
   extern __shared__ __align__(16) unsigned char sm[];
   const int r = blockIdx.x / p.G;
   const int kb = blockIdx.x - r * p.G;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-  const uint64_t kdim = p.kdim, nvec = p.hidden / 8, ntiles = p.hidden / 16, pairs = kdim / 32;
+  const uint64_t kdim = p.kdim, nvec = p.hidden / 8, ntiles = p.hidden / 16;
   const uint32_t per = p.per_cta, ks = p.ks, tokens = p.tokens;
   const uint32_t epoch = p.epoch_dev != nullptr ? device_epoch(p.epoch_dev) : p.epoch;
   if (epoch == 0 || epoch == 0xFFFFFFFFu) {  // device epochs ran out: sfc_reset first
@@ -264,38 +287,85 @@ __global__ void __launch_bounds__(kLinearThreads, 2) linear_mma_kernel(const __g
   uint4* ownv = reinterpret_cast<uint4*>(parts + static_cast<uint64_t>(per) * ks * 128);
   uint32_t* cnt = reinterpret_cast<uint32_t*>(ownv + static_cast<uint64_t>(per) * 16);
 
-  copy_to_smem_async(xs, p.x[r], static_cast<uint64_t>(tokens) * kdim * 2);
+  // x_r into shared memory: every thread issues its 16-byte asynchronous
+  // copies (no register round trip) before any is waited for, so the whole
+  // activation is in flight at once
+  {
+    const uint32_t xb = static_cast<uint32_t>(__cvta_generic_to_shared(xs));
+    const char* src = reinterpret_cast<const char*>(p.x[r]);
+    const uint32_t bytes = static_cast<uint32_t>(tokens * kdim * 2);
+#pragma unroll 1
+    for (uint32_t o = threadIdx.x * 16; o < bytes; o += kLinearThreads * 16)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(xb + o), "l"(src + o) : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+
+  const uint32_t groups = kLinearWarps / ks, grp = warp / ks, h = warp % ks;
+  const uint64_t blocks = kdim / B::kCols;                                // whole blocks of a row
+  const bool rest32 = kWide && (kdim & 63) != 0 && h == ks - 1;          // this part takes the 32-column rest
+  const uint64_t s_lo = blocks * h / ks, s_hi = blocks * (h + 1) / ks;  // this warp's blocks
+  const uint64_t ring_end = s_lo + (s_hi - s_lo) / kRing * kRing;        // blocks that go through the ring
+  const bool ring = ring_end > s_lo;
+  const uint16_t* W = p.W[r];
+  const uint32_t col = q * (B::kCols / 4);  // the thread's first column in a block
+  uint32_t a[kRing][B::kRegs], b[kRing][B::kRegs];
+  bool filled = false;  // the ring holds the first tile's first kRing blocks
+  if (ring && grp < owned) {
+    const uint16_t* wg = W + ((t0 + grp) * 16 + g) * kdim + col;
+#pragma unroll
+    for (int i = 0; i < kRing; ++i) {
+      B::load(wg + (s_lo + i) * B::kCols, a[i]);
+      B::load(wg + 8 * kdim + (s_lo + i) * B::kCols, b[i]);
+    }
+    filled = true;
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
   for (uint32_t i = threadIdx.x; i < per; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
 
-  const uint32_t groups = kLinearWarps / ks, grp = warp / ks, h = warp % ks;
-  const uint64_t s_lo = pairs * h / ks, s_hi = pairs * (h + 1) / ks;  // this warp's 32-column blocks
-  const uint16_t* W = p.W[r];
   const bool tok_ok = static_cast<uint32_t>(g) < tokens;
-  const uint16_t* xrow = xs + (tok_ok ? g : 0) * kdim + 8 * q;
+  const uint16_t* xrow = xs + (tok_ok ? g : 0) * kdim + col;
   for (uint32_t t = grp; t < owned; t += groups) {
-    const uint16_t* wg = W + ((t0 + t) * 16 + g) * kdim + 8 * q;  // row g; row g + 8 is 8 kdim further
+    const uint16_t* wg = W + ((t0 + t) * 16 + g) * kdim + col;  // row g; row g + 8 is 8 kdim further
     float d[4] = {0.f, 0.f, 0.f, 0.f};
     uint64_t s = s_lo;
-    for (; s + kMmaPairs <= s_hi; s += kMmaPairs) {
-      uint4 a[kMmaPairs], b[kMmaPairs];
+    if (ring) {
+      if (!filled) {
 #pragma unroll
-      for (int i = 0; i < kMmaPairs; ++i) {
-        a[i] = ld_stream_v4(wg + (s + i) * 32);
-        b[i] = ld_stream_v4(wg + 8 * kdim + (s + i) * 32);
+        for (int i = 0; i < kRing; ++i) {
+          B::load(wg + (s_lo + i) * B::kCols, a[i]);
+          B::load(wg + 8 * kdim + (s_lo + i) * B::kCols, b[i]);
+        }
+      }
+      for (; s + kRing < ring_end; s += kRing) {
+#pragma unroll
+        for (int i = 0; i < kRing; ++i) {
+          B::mma(d, a[i], b[i], xrow + (s + i) * B::kCols, tok_ok);
+          B::load(wg + (s + kRing + i) * B::kCols, a[i]);
+          B::load(wg + 8 * kdim + (s + kRing + i) * B::kCols, b[i]);
+        }
       }
 #pragma unroll
-      for (int i = 0; i < kMmaPairs; ++i) {
-        const uint4 xv = tok_ok ? *reinterpret_cast<const uint4*>(xrow + (s + i) * 32) : make_uint4(0, 0, 0, 0);
-        mma_16x8x16(d, a[i].x, b[i].x, a[i].y, b[i].y, xv.x, xv.y);
-        mma_16x8x16(d, a[i].z, b[i].z, a[i].w, b[i].w, xv.z, xv.w);
+      for (int i = 0; i < kRing; ++i) {
+        B::mma(d, a[i], b[i], xrow + (s + i) * B::kCols, tok_ok);
       }
+      filled = false;
+      s = ring_end;
     }
     for (; s < s_hi; ++s) {
-      const uint4 a = ld_stream_v4(wg + s * 32), b = ld_stream_v4(wg + 8 * kdim + s * 32);
-      const uint4 xv = tok_ok ? *reinterpret_cast<const uint4*>(xrow + s * 32) : make_uint4(0, 0, 0, 0);
-      mma_16x8x16(d, a.x, b.x, a.y, b.y, xv.x, xv.y);
-      mma_16x8x16(d, a.z, b.z, a.w, b.w, xv.z, xv.w);
+      uint32_t a1[B::kRegs], b1[B::kRegs];
+      B::load(wg + s * B::kCols, a1);
+      B::load(wg + 8 * kdim + s * B::kCols, b1);
+      B::mma(d, a1, b1, xrow + s * B::kCols, tok_ok);
+    }
+    if (rest32) {  // columns blocks * 64 .. + 31 as one 16-byte-piece block (thread columns 8q .. 8q+7)
+      using R = MmaBlock<false>;
+      const uint64_t c0 = blocks * 64 + 8 * q;
+      const uint16_t* wt = W + ((t0 + t) * 16 + g) * kdim + c0;
+      uint32_t a1[R::kRegs], b1[R::kRegs];
+      R::load(wt, a1);
+      R::load(wt + 8 * kdim, b1);
+      R::mma(d, a1, b1, xs + (tok_ok ? g : 0) * kdim + c0, tok_ok);
     }
     // d0, d1: row g, tokens 2q, 2q+1; d2, d3: row g + 8, same tokens
     float* pt = parts + (static_cast<uint64_t>(t) * ks + h) * 128;
@@ -348,9 +418,10 @@ __global__ void __launch_bounds__(kLinearThreads, 2) linear_mma_kernel(const __g
 
 template <int NR>
 struct LinearRow {
-  static const void* get(uint32_t T) {
-    switch (T) {
-      case 0: return reinterpret_cast<const void*>(&linear_mma_kernel<NR>);  // tensor-core tile
+  static const void* get(uint32_t variant) {
+    switch (variant) {
+      case kLinearMma16: return reinterpret_cast<const void*>(&linear_mma_kernel<NR, false>);
+      case kLinearMma32: return reinterpret_cast<const void*>(&linear_mma_kernel<NR, true>);
       case 1: return reinterpret_cast<const void*>(&linear_allreduce_kernel<NR, 1>);
       case 2: return reinterpret_cast<const void*>(&linear_allreduce_kernel<NR, 2>);
       case 4: return reinterpret_cast<const void*>(&linear_allreduce_kernel<NR, 4>);
@@ -362,15 +433,15 @@ struct LinearRow {
 
 }  // namespace
 
-const void* linear_kernel_for(int nranks, uint32_t token_tile) {
+const void* linear_kernel_for(int nranks, uint32_t variant) {
   switch (nranks) {
-    case 2: return LinearRow<2>::get(token_tile);
-    case 3: return LinearRow<3>::get(token_tile);
-    case 4: return LinearRow<4>::get(token_tile);
-    case 5: return LinearRow<5>::get(token_tile);
-    case 6: return LinearRow<6>::get(token_tile);
-    case 7: return LinearRow<7>::get(token_tile);
-    case 8: return LinearRow<8>::get(token_tile);
+    case 2: return LinearRow<2>::get(variant);
+    case 3: return LinearRow<3>::get(variant);
+    case 4: return LinearRow<4>::get(variant);
+    case 5: return LinearRow<5>::get(variant);
+    case 6: return LinearRow<6>::get(variant);
+    case 7: return LinearRow<7>::get(variant);
+    case 8: return LinearRow<8>::get(variant);
     default: return nullptr;
   }
 }

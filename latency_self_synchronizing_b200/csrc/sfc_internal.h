@@ -38,8 +38,10 @@ constexpr int kSentinelLoadPoll = 16;
 // it one atomic exchange per unit has the lower latency; above it the
 // exchanges queue on the L2's atomic units (measured on B200: at 8 ranks
 // x 128 KB p50 5.5 -> 3.5 us, p99 15 -> 4 us; at 4 ranks x 16 KB the
-// exchange is 0.35 us faster).
-constexpr uint64_t kSentinelLoadPollBytes = 448 * 1024;
+// exchange is 0.35 us faster). At 4 ranks x 128 KB, the point itself, the
+// loads trade 4 % of p50 (2.18 -> 2.27 us) and 2 % of the mean for a 16 %
+// lower p99 (3.1-3.2 -> 2.7 us).
+constexpr uint64_t kSentinelLoadPollBytes = 384 * 1024;
 inline bool sentinel_load_poll(int n, uint64_t count) {
   return static_cast<uint64_t>(n - 1) * count * 2 >= kSentinelLoadPollBytes;
 }
@@ -140,13 +142,19 @@ inline uint32_t linear_token_tile(uint32_t tokens) { return tokens <= 1 ? 1 : to
 inline size_t linear_smem_bytes(uint64_t kdim, uint32_t T, uint32_t ks, uint32_t per_cta) {
   return kdim * 2 * T + 32ull * ks * T * per_cta + 16ull * T * per_cta + 4ull * per_cta;
 }
-// tensor-core kernel (2..8 tokens, 16-row tiles): x, per-part sums of 16 x 8,
-// own vectors (2 x 8 per tile), counters
+// The tensor-core kernels (2..8 tokens, 16-row tiles) read each weight row
+// as 16-byte pieces (32-column blocks) or as 32-byte pieces (64-column
+// blocks; the weights 32-byte aligned).
+constexpr uint32_t kLinearMma16 = 0;
+constexpr uint32_t kLinearMma32 = 32;
+// tensor-core kernel: x, per-part sums of 16 x 8, own vectors (2 x 8 per
+// tile), counters
 inline size_t linear_mma_smem_bytes(uint64_t kdim, uint32_t tokens, uint32_t ks, uint32_t per_tiles) {
   return ((tokens * kdim * 2 + 15) & ~15ull) + 512ull * ks * per_tiles + 256ull * per_tiles + 4ull * per_tiles;
 }
-// token_tile 1, 2, 4, 8: the CUDA-core kernel; 0: the tensor-core kernel
-const void* linear_kernel_for(int nranks, uint32_t token_tile);
+// variant 1, 2, 4, 8: the CUDA-core kernel of that token tile;
+// kLinearMma16 / kLinearMma32: a tensor-core kernel
+const void* linear_kernel_for(int nranks, uint32_t variant);
 
 // Kernel entry for (nranks, protocol, op); null if not provided.
 const void* kernel_for(int nranks, int protocol, int op);

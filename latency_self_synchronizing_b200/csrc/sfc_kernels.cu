@@ -334,7 +334,7 @@ SFC_DEV bool sentinel_poll(const KParams& p, int r, int op, uint64_t gtid, uint6
 //    release fence. A writer reuses the slot two epochs later only after it
 //    has seen this rank's next push (its poll followed by its own acquire
 //    fence), so the release / acquire pair orders the resets before that
-//    reuse. No atomics: at (N - 1) x bytes >= 448 KB the L2's atomic
+//    reuse. No atomics: at (N - 1) x bytes >= 384 KB the L2's atomic
 //    throughput, not the round trip, bounds the exchange polls, and the
 //    release fence (about 0.5 us) costs less than the atomics it saves.
 template <int N, int OP, bool kLoadPoll>

@@ -48,7 +48,7 @@ struct sfc_ctx {
                                                // variant), 0 = unknown
   int forced_protocol = 0;                // SFC_PROTOCOL: what AUTO resolves to (0 = the selector)
   int smem_optin = 0;                     // opt-in shared memory per block (bytes)
-  int linear_occ[5] = {};                 // fused-linear CTAs per SM: token tile 1/2/4/8, tensor-core (0 = not queried)
+  int linear_occ[5] = {};                 // fused-linear CTAs per SM: token tile 1/2/4/8, tensor cores (0 = not queried)
 
   // staging for the host-buffer entry point, and the copy streams and
   // events that overlap its copies with the chain segments
@@ -858,7 +858,7 @@ sfc_status sfc_linear_allreduce_tokens(sfc_ctx* c, const void* const* W, const v
   // cores (16-row x 8-token tiles); one token, or other shapes, on the CUDA
   // cores (token tile T)
   const bool mma = tokens >= 2 && hidden % 16 == 0 && kdim % 32 == 0;
-  const uint32_t T = mma ? 0 : sfc::linear_token_tile(tokens);
+  const uint32_t T = mma ? kLinearMma16 : sfc::linear_token_tile(tokens);
   if (hidden == 0 || hidden % 8 || hidden * tokens > c->max_count || kdim == 0 || kdim % 8 ||
       kdim * (mma ? tokens : T) > 49152)
     return SFC_ERR_INVALID;
@@ -882,7 +882,13 @@ sfc_status sfc_linear_allreduce_tokens(sfc_ctx* c, const void* const* W, const v
       if (overlap(y[a], yb, x[b], xb) || overlap(y[a], yb, W[b], hidden * kdim * 2) ||
           (a < b && overlap(y[a], yb, y[b], yb)))
         return SFC_ERR_INVALID;
-  const void* fn = linear_kernel_for(N, T);
+  // The tensor-core kernels: 32-byte weight pieces where ks >= 2 warps share
+  // a tile (measured on B200: 0.92-0.97 of the weight stream there against
+  // 0.75-0.87 with 16-byte pieces), 16-byte pieces where every warp owns
+  // whole tiles (2-5 % faster there). 32-byte loads need every W_r 32-byte
+  // aligned; otherwise the 16-byte pieces serve every shape.
+  bool w32_ok = mma;
+  for (int r = 0; r < N && w32_ok; ++r) w32_ok = (reinterpret_cast<uintptr_t>(W[r]) & 31u) == 0;
   // as many CTAs per rank as fit (two per SM), each rank's output units
   // (8-row vectors, or 16-row tiles on the tensor cores) split evenly over
   // its CTAs; ks warps share a unit when that evens out the 8 warps' work
@@ -892,14 +898,22 @@ sfc_status sfc_linear_allreduce_tokens(sfc_ctx* c, const void* const* W, const v
   const int ti = mma ? 4 : T == 1 ? 0 : T == 2 ? 1 : T == 4 ? 2 : 3;
   int occ = c->linear_occ[ti];
   if (occ == 0) {
-    if (!cuda_ok(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, c->smem_optin)))
-      return SFC_ERR_CUDA;
-    if (!cuda_ok(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kLinearThreads, 0)) || occ < 1)
-      return SFC_ERR_RESOURCES;
-    c->linear_occ[ti] = occ = std::min(occ, 2);
+    occ = 2;
+    for (const uint32_t v : {T, mma ? kLinearMma32 : T}) {  // both tensor-core kernels share the cache entry
+      const void* f = linear_kernel_for(N, v);
+      int o = 0;
+      if (f == nullptr) return SFC_ERR_UNSUPPORTED;
+      if (!cuda_ok(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, c->smem_optin)))
+        return SFC_ERR_CUDA;
+      if (!cuda_ok(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, f, kLinearThreads, 0)) || o < 1)
+        return SFC_ERR_RESOURCES;
+      occ = std::min(occ, o);
+    }
+    c->linear_occ[ti] = occ;
   }
   int G = occ * c->sm_count / N;
   uint32_t per = 0, ks = 1;
+  bool wide = false;
   for (;; --G) {
     if (G < 1) return SFC_ERR_RESOURCES;
     per = static_cast<uint32_t>((units + G - 1) / G);
@@ -913,6 +927,7 @@ sfc_status sfc_linear_allreduce_tokens(sfc_ctx* c, const void* const* W, const v
         ks = cand;
       }
     }
+    wide = w32_ok && ks >= 2;
     // both CTAs of an SM must fit: fewer, larger CTAs if not
     const size_t smem =
         mma ? sfc::linear_mma_smem_bytes(kdim, tokens, ks, per) : sfc::linear_smem_bytes(kdim, T, ks, per);
@@ -922,6 +937,7 @@ sfc_status sfc_linear_allreduce_tokens(sfc_ctx* c, const void* const* W, const v
   }
   const int smem = static_cast<int>(mma ? sfc::linear_mma_smem_bytes(kdim, tokens, ks, per)
                                          : sfc::linear_smem_bytes(kdim, T, ks, per));
+  const void* fn = linear_kernel_for(N, wide ? kLinearMma32 : T);
   p.per_cta = per;
   p.ks = ks;
   p.hidden = hidden;

@@ -78,13 +78,16 @@ def test_linear_allreduce_shares_the_epoch_sequence():
         comm.close()
 
 
-# several decode tokens in one pass over the weights: 1-2 tokens (and ragged
-# shapes) on the CUDA cores with token tiles 2, 4, 8 (extra tokens masked),
-# 3-8 tokens on 16-aligned shapes on the tensor cores (16 x 8 tiles)
+# several decode tokens in one pass over the weights: ragged shapes on the
+# CUDA cores with token tiles 2, 4, 8 (extra tokens masked), 2-8 tokens on
+# 16-aligned shapes on the tensor cores (16 x 8 tiles): 16-byte weight pieces
+# where each warp owns whole tiles, 32-byte pieces where 2-4 warps share one
+# (4 x 512 x 4096, 4 x 4096 x 2048, and 2 x 256 x 2080 with its 32-column rest)
 @pytest.mark.parametrize("n,hidden,kdim,tokens", [(2, 64, 512, 2), (4, 8192, 3584, 4), (8, 1024, 1024, 8),
                                                   (3, 2056, 136, 3), (4, 512, 4096, 5), (2, 1000, 2048, 7),
                                                   (8, 64, 8, 6), (5, 8192, 1024, 8), (3, 2064, 144, 3),
-                                                  (4, 4096, 2048, 2), (3, 2064, 160, 3), (2, 1000, 512, 2)])
+                                                  (4, 4096, 2048, 2), (3, 2064, 160, 3), (2, 1000, 512, 2),
+                                                  (2, 256, 2080, 3)])
 def test_linear_allreduce_tokens_within_bound(n, hidden, kdim, tokens):
     w, _ = _case(n, hidden, kdim, seed=hidden * 3 + kdim + n + tokens)
     x = make_inputs(seed=hidden + tokens, k_ops=1, nranks=n, count=tokens * kdim, dist="normal",
@@ -105,5 +108,37 @@ def test_linear_allreduce_tokens_within_bound(n, hidden, kdim, tokens):
             bound = linear.linear_allreduce_error_bound(w, x)
             got = bf16_bits_to_f32(ys[0]).reshape(tokens, hidden).astype(np.float64)
             assert np.all(np.abs(got - exact) <= bound)
+    finally:
+        comm.close()
+
+
+def test_linear_allreduce_tokens_weights_16_byte_aligned():
+    """Weights that start 16 bytes past a 32-byte boundary take the 16-byte
+    pieces on a shape that otherwise reads 32-byte pieces; same bound."""
+    n, hidden, kdim, tokens = 4, 4096, 2048, 2
+    w, _ = _case(n, hidden, kdim, seed=77)
+    x = make_inputs(seed=78, k_ops=1, nranks=n, count=tokens * kdim, dist="normal",
+                    params=(1.0,))[0].reshape(n, tokens, kdim)
+    comm = api.Communicator(n, tokens * hidden * 2, protocols=["ll"])
+    try:
+        W = []
+        for r in range(n):
+            big = torch.empty(hidden * kdim + 8, dtype=torch.bfloat16, device="cuda")
+            assert big.data_ptr() % 32 == 0
+            view = big[8:].view(hidden, kdim)  # 16 bytes in
+            view.copy_(_bf16_dev(w[r]).view(hidden, kdim))
+            W.append(view)
+        X = [_bf16_dev(x[r]) for r in range(n)]
+        Y = [torch.empty(tokens, hidden, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+        comm.linear_allreduce(W, X, Y)
+        torch.cuda.synchronize()
+        assert comm.status()[0] == api.Status.OK
+        ys = [Y[r].cpu().view(torch.int16).numpy().view(np.uint16) for r in range(n)]
+        for r in range(1, n):
+            np.testing.assert_array_equal(ys[r], ys[0])
+        exact = linear.linear_allreduce_fp64(w, x)
+        bound = linear.linear_allreduce_error_bound(w, x)
+        got = bf16_bits_to_f32(ys[0]).reshape(tokens, hidden).astype(np.float64)
+        assert np.all(np.abs(got - exact) <= bound)
     finally:
         comm.close()

@@ -76,9 +76,10 @@ def test_odd_rank_counts_under_skew(proto, n):
     _run(proto, n=n, count=777, total_ops=1 << 15, skew_mean_ns=500.0, seed=20 + n)
 
 
-@pytest.mark.parametrize("n,count", [(8, 32769), (4, 80000), (2, 262147)])
+@pytest.mark.parametrize("n,count", [(8, 32769), (4, 80000), (4, 65536), (2, 262147)])
 def test_sentinel_load_polls_under_skew(n, count):
-    """Large sentinel messages ((N - 1) x bytes >= 448 KB) poll with loads and
-    reset with stores behind a release fence: the resets must land before a
-    writer reuses the slot two epochs later, under changing arrival orders."""
+    """Large sentinel messages ((N - 1) x bytes >= 384 KB; 4 x 128 KB is the
+    smallest power-of-two case) poll with loads and reset with stores behind
+    a release fence: the resets must land before a writer reuses the slot two
+    epochs later, under changing arrival orders."""
     _run("sentinel", n=n, count=count, total_ops=1 << 13, skew_mean_ns=2000.0, seed=30 + n)
