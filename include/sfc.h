@@ -379,10 +379,13 @@ sfc_status sfc_linear_allreduce(sfc_ctx* ctx, const void* const* W, const void* 
  * all tokens and the all-reduce covers tokens * hidden elements (one epoch).
  * tokens * hidden <= max count of the context; kdim * T <= 49152, T = tokens
  * rounded up to 1, 2, 4 or 8; 2+ tokens with hidden % 16 == 0 and
- * kdim % 32 == 0 run on the tensor cores instead, with tokens * kdim <= 49152.
+ * kdim % 32 == 0 run on the tensor cores instead, with tokens * kdim <= 49152
+ * (where several warps share a tile's columns, weights that are 32-byte
+ * aligned are read in 32-byte pieces, otherwise in 16-byte pieces).
  * sfc_linear_allreduce is tokens = 1. Measured on B200 against a library
- * tensor-core GEMM + all-reduce: 1.07-1.16x faster at 1-4 tokens, equal to
- * 1.13x faster at 8. */
+ * tensor-core GEMM + all-reduce on 8192-hidden shapes: 1.06-1.23x faster at
+ * 2-8 tokens; within 3 % of it on the largest shapes; slower (0.78x) where
+ * the activation fills most of the shared memory (2 x 8192 x 6144 x 8). */
 sfc_status sfc_linear_allreduce_tokens(sfc_ctx* ctx, const void* const* W, const void* const* x, void* const* y,
                                        size_t hidden, size_t kdim, uint32_t tokens, uint32_t epoch, void* stream);
 
