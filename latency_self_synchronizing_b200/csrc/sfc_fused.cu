@@ -227,7 +227,7 @@ template <bool kWide>
 struct MmaBlock {
   static constexpr int kCols = kWide ? 64 : 32;  // columns per block
   static constexpr int kRegs = kWide ? 8 : 4;    // registers per row piece
-  static constexpr int kRing = kWide ? 4 : 8;    // blocks in flight per thread: 256 bytes either way
+  static constexpr int kRing = kWide ? 4 : 8;    // blocks in flight per thread: 256 bytes either way (x2 at one CTA an SM)
   SFC_DEV static void load(const uint16_t* src, uint32_t (&v)[kRegs]) {
     if constexpr (kWide) {
       ld_stream_v8(src, v);
@@ -259,11 +259,14 @@ struct MmaBlock {
 // during a tile's last round, and x rows padded to shift the token rows'
 // banks, each 0.5-2 % slower.) With 32-byte pieces a 32-column rest of the
 // row (kdim % 64 == 32) is one 16-byte-piece block, taken by the tile's last
-// part.
-template <int NR, bool kWide>
-__global__ void __launch_bounds__(kLinearThreads, 2) linear_mma_kernel(const __grid_constant__ LinearParams p) {
+// part. kCtasPerSm = 1: one CTA an SM with a ring twice as deep (the same
+// bytes in flight an SM), for activations so large that two CTAs' shared
+// memory would leave the SM's unified L1 too little room for the loads in
+// flight.
+template <int NR, bool kWide, int kCtasPerSm>
+__global__ void __launch_bounds__(kLinearThreads, kCtasPerSm) linear_mma_kernel(const __grid_constant__ LinearParams p) {
   using B = MmaBlock<kWide>;
-  constexpr int kRing = B::kRing;
+  constexpr int kRing = B::kRing * (kCtasPerSm == 1 ? 2 : 1);
   extern __shared__ __align__(16) unsigned char sm[];
   const int r = blockIdx.x / p.G;
   const int kb = blockIdx.x - r * p.G;
@@ -420,8 +423,12 @@ template <int NR>
 struct LinearRow {
   static const void* get(uint32_t variant) {
     switch (variant) {
-      case kLinearMma16: return reinterpret_cast<const void*>(&linear_mma_kernel<NR, false>);
-      case kLinearMma32: return reinterpret_cast<const void*>(&linear_mma_kernel<NR, true>);
+      case kLinearMma16: return reinterpret_cast<const void*>(&linear_mma_kernel<NR, false, 2>);
+      case kLinearMma32: return reinterpret_cast<const void*>(&linear_mma_kernel<NR, true, 2>);
+      case kLinearMma16 + kLinearMmaOnePerSm:
+        return reinterpret_cast<const void*>(&linear_mma_kernel<NR, false, 1>);
+      case kLinearMma32 + kLinearMmaOnePerSm:
+        return reinterpret_cast<const void*>(&linear_mma_kernel<NR, true, 1>);
       case 1: return reinterpret_cast<const void*>(&linear_allreduce_kernel<NR, 1>);
       case 2: return reinterpret_cast<const void*>(&linear_allreduce_kernel<NR, 2>);
       case 4: return reinterpret_cast<const void*>(&linear_allreduce_kernel<NR, 4>);

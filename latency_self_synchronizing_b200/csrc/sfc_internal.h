@@ -147,13 +147,17 @@ inline size_t linear_smem_bytes(uint64_t kdim, uint32_t T, uint32_t ks, uint32_t
 // blocks; the weights 32-byte aligned).
 constexpr uint32_t kLinearMma16 = 0;
 constexpr uint32_t kLinearMma32 = 32;
+// added to either: one CTA an SM with a ring twice as deep
+constexpr uint32_t kLinearMmaOnePerSm = 64;
+// shared memory per CTA above which two CTAs an SM give way to one
+constexpr size_t kLinearOnePerSmSmemBytes = 96 * 1024;
 // tensor-core kernel: x, per-part sums of 16 x 8, own vectors (2 x 8 per
 // tile), counters
 inline size_t linear_mma_smem_bytes(uint64_t kdim, uint32_t tokens, uint32_t ks, uint32_t per_tiles) {
   return ((tokens * kdim * 2 + 15) & ~15ull) + 512ull * ks * per_tiles + 256ull * per_tiles + 4ull * per_tiles;
 }
 // variant 1, 2, 4, 8: the CUDA-core kernel of that token tile;
-// kLinearMma16 / kLinearMma32: a tensor-core kernel
+// kLinearMma16 / kLinearMma32 (+ kLinearMmaOnePerSm): a tensor-core kernel
 const void* linear_kernel_for(int nranks, uint32_t variant);
 
 // Kernel entry for (nranks, protocol, op); null if not provided.

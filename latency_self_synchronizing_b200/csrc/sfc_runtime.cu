@@ -49,6 +49,7 @@ struct sfc_ctx {
   int forced_protocol = 0;                // SFC_PROTOCOL: what AUTO resolves to (0 = the selector)
   int smem_optin = 0;                     // opt-in shared memory per block (bytes)
   int linear_occ[5] = {};                 // fused-linear CTAs per SM: token tile 1/2/4/8, tensor cores (0 = not queried)
+  int linear_occ_one = 0;                 // the one-CTA-per-SM tensor-core kernels: set up (1) or not (0)
 
   // staging for the host-buffer entry point, and the copy streams and
   // events that overlap its copies with the chain segments
@@ -911,33 +912,58 @@ sfc_status sfc_linear_allreduce_tokens(sfc_ctx* c, const void* const* W, const v
     }
     c->linear_occ[ti] = occ;
   }
-  int G = occ * c->sm_count / N;
+  int G = 0;
   uint32_t per = 0, ks = 1;
   bool wide = false;
-  for (;; --G) {
-    if (G < 1) return SFC_ERR_RESOURCES;
-    per = static_cast<uint32_t>((units + G - 1) / G);
-    double best = -1.0;
-    for (uint32_t cand = 1; cand <= 8; cand *= 2) {
-      if (cand > 1 && kparts < cand) break;
-      const uint32_t groups = 8 / cand, rounds = (per + groups - 1) / groups;
-      const double eff = static_cast<double>(per) / (static_cast<double>(rounds) * groups);
-      if (eff > best + 1e-9) {
-        best = eff;
-        ks = cand;
+  size_t smem = 0;
+  // G, per, ks, piece width and shared memory from G0 CTAs per rank down
+  // until the CTAs fit (both CTAs of an SM when two share one)
+  auto fit = [&](int G0) {
+    for (G = G0; G >= 1; --G) {
+      per = static_cast<uint32_t>((units + G - 1) / G);
+      double best = -1.0;
+      for (uint32_t cand = 1; cand <= 8; cand *= 2) {
+        if (cand > 1 && kparts < cand) break;
+        const uint32_t groups = 8 / cand, rounds = (per + groups - 1) / groups;
+        const double eff = static_cast<double>(per) / (static_cast<double>(rounds) * groups);
+        if (eff > best + 1e-9) {
+          best = eff;
+          ks = cand;
+        }
       }
+      wide = w32_ok && ks >= 2;
+      smem = mma ? sfc::linear_mma_smem_bytes(kdim, tokens, ks, per) : sfc::linear_smem_bytes(kdim, T, ks, per);
+      if (smem <= static_cast<size_t>(c->smem_optin) &&
+          (G * N <= c->sm_count || 2 * (smem + 1024) <= static_cast<size_t>(c->smem_optin) + 1024))
+        return true;
     }
-    wide = w32_ok && ks >= 2;
-    // both CTAs of an SM must fit: fewer, larger CTAs if not
-    const size_t smem =
-        mma ? sfc::linear_mma_smem_bytes(kdim, tokens, ks, per) : sfc::linear_smem_bytes(kdim, T, ks, per);
-    if (smem <= static_cast<size_t>(c->smem_optin) &&
-        (G * N <= c->sm_count || 2 * (smem + 1024) <= static_cast<size_t>(c->smem_optin) + 1024))
-      break;
+    return false;
+  };
+  if (!fit(occ * c->sm_count / N)) return SFC_ERR_RESOURCES;
+  // Two CTAs an SM whose shared memory passes 2 x 96 KB leave the SM's
+  // unified L1 too little room for the weight loads in flight; where the SMs
+  // divide evenly among the ranks, one CTA an SM with a ring twice as deep
+  // keeps the same bytes in flight and holds x once (measured on B200,
+  // 2 x 8192 x 6144 x 8 tokens: 51.6 -> 34.9 us; at 56-86 KB of x, one CTA an
+  // SM was 4-12 % slower, so it stays off there).
+  bool one_per_sm = false;
+  if (mma && c->sm_count % N == 0 && smem > kLinearOnePerSmSmemBytes) {
+    if (c->linear_occ_one == 0) {
+      for (const uint32_t v : {kLinearMma16 + kLinearMmaOnePerSm, kLinearMma32 + kLinearMmaOnePerSm}) {
+        const void* f = linear_kernel_for(N, v);
+        int o = 0;
+        if (f == nullptr) return SFC_ERR_UNSUPPORTED;
+        if (!cuda_ok(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, c->smem_optin)))
+          return SFC_ERR_CUDA;
+        if (!cuda_ok(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, f, kLinearThreads, 0)) || o < 1)
+          return SFC_ERR_RESOURCES;
+      }
+      c->linear_occ_one = 1;
+    }
+    one_per_sm = true;
+    if (!fit(c->sm_count / N)) return SFC_ERR_RESOURCES;
   }
-  const int smem = static_cast<int>(mma ? sfc::linear_mma_smem_bytes(kdim, tokens, ks, per)
-                                         : sfc::linear_smem_bytes(kdim, T, ks, per));
-  const void* fn = linear_kernel_for(N, wide ? kLinearMma32 : T);
+  const void* fn = linear_kernel_for(N, (wide ? kLinearMma32 : T) + (one_per_sm ? kLinearMmaOnePerSm : 0u));
   p.per_cta = per;
   p.ks = ks;
   p.hidden = hidden;

@@ -82,12 +82,15 @@ def test_linear_allreduce_shares_the_epoch_sequence():
 # CUDA cores with token tiles 2, 4, 8 (extra tokens masked), 2-8 tokens on
 # 16-aligned shapes on the tensor cores (16 x 8 tiles): 16-byte weight pieces
 # where each warp owns whole tiles, 32-byte pieces where 2-4 warps share one
-# (4 x 512 x 4096, 4 x 4096 x 2048, and 2 x 256 x 2080 with its 32-column rest)
+# (4 x 512 x 4096, 4 x 4096 x 2048, and 2 x 256 x 2080 with its 32-column rest);
+# a 96 KB activation at 2 and 4 ranks takes one CTA an SM (2 x 512 x 6144 on
+# 32-byte pieces, 4 x 3584 x 6144 on 16-byte pieces)
 @pytest.mark.parametrize("n,hidden,kdim,tokens", [(2, 64, 512, 2), (4, 8192, 3584, 4), (8, 1024, 1024, 8),
                                                   (3, 2056, 136, 3), (4, 512, 4096, 5), (2, 1000, 2048, 7),
                                                   (8, 64, 8, 6), (5, 8192, 1024, 8), (3, 2064, 144, 3),
                                                   (4, 4096, 2048, 2), (3, 2064, 160, 3), (2, 1000, 512, 2),
-                                                  (2, 256, 2080, 3)])
+                                                  (2, 256, 2080, 3), (2, 512, 6144, 8),
+                                                  (4, 3584, 6144, 8)])
 def test_linear_allreduce_tokens_within_bound(n, hidden, kdim, tokens):
     w, _ = _case(n, hidden, kdim, seed=hidden * 3 + kdim + n + tokens)
     x = make_inputs(seed=hidden + tokens, k_ops=1, nranks=n, count=tokens * kdim, dist="normal",
