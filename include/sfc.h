@@ -384,8 +384,7 @@ sfc_status sfc_linear_allreduce(sfc_ctx* ctx, const void* const* W, const void* 
  * aligned are read in 32-byte pieces, otherwise in 16-byte pieces).
  * sfc_linear_allreduce is tokens = 1. Measured on B200 against a library
  * tensor-core GEMM + all-reduce on 8192-hidden shapes: 1.06-1.23x faster at
- * 2-8 tokens; within 3 % of it on the largest shapes; slower (0.78x) where
- * the activation fills most of the shared memory (2 x 8192 x 6144 x 8). */
+ * 2-8 tokens; within 3 % of it on the largest shapes. */
 sfc_status sfc_linear_allreduce_tokens(sfc_ctx* ctx, const void* const* W, const void* const* x, void* const* y,
                                        size_t hidden, size_t kdim, uint32_t tokens, uint32_t epoch, void* stream);
 
