@@ -27,7 +27,9 @@
 // kernel instance carries a token tile T (1, 2, 4 or 8), keeps 8 x T dot
 // products per lane and pushes one vector per (token, 8 rows); token u's
 // vector v is LL vector u * hidden / 8 + v, so the all-reduce covers
-// tokens x hidden elements.
+// tokens x hidden elements. Shapes in whole 16-row, 32-column tiles take the
+// tensor-core kernels below instead for 2..8 tokens (16-row x 8-token MMA
+// tiles, weight pieces of 16 or 32 bytes, one or two CTAs an SM).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
