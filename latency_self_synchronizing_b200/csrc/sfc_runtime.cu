@@ -100,7 +100,9 @@ bool overlap(const void* a, size_t n, const void* b, size_t m) {
 // work over twice as many 128-thread CTAs (fewer polls in flight per SM):
 // 5-13 % lower latency at 8 ranks and 8-64 KB, equal or better at 4 ranks,
 // measured on B200 for LL, sentinel and the one-load LL128. Everything else
-// keeps kThreads. A caller-fixed CTA count keeps kThreads too.
+// keeps kThreads. A caller-fixed CTA count keeps kThreads too. (64-thread
+// CTAs up to 16 KB measured slower at 4 ranks, 4 x 16 KB sentinel 1.70-1.73
+// -> 1.79 us, and from 3 % faster to 25 % slower at 8 ranks: not used.)
 int cta_threads(const sfc_ctx* c, int proto, uint64_t count) {
   const bool small_msg = c->nranks >= 4 && count <= kSmallCtaMaxCount && c->cfg.ctas_per_rank == 0;
   return small_msg && (proto == kLL || proto == kSentinel || proto == kLL128Fast) ? kSmallCtaThreads : kThreads;
