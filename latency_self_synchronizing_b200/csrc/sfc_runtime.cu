@@ -902,8 +902,9 @@ sfc_status sfc_linear_allreduce_tokens(sfc_ctx* c, const void* const* W, const v
   int occ = c->linear_occ[ti];
   if (occ == 0) {
     occ = 2;
-    for (const uint32_t v : {T, mma ? kLinearMma32 : T}) {  // both tensor-core kernels share the cache entry
-      const void* f = linear_kernel_for(N, v);
+    const uint32_t kernels[2] = {T, kLinearMma32};  // both tensor-core kernels share the cache entry
+    for (int k = 0; k < (mma ? 2 : 1); ++k) {
+      const void* f = linear_kernel_for(N, kernels[k]);
       int o = 0;
       if (f == nullptr) return SFC_ERR_UNSUPPORTED;
       if (!cuda_ok(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, c->smem_optin)))
